@@ -1,0 +1,425 @@
+// api.cu -- the C ABI of libdsa (declared in include/dsa.h): argument
+// validation, workspace layout, TMA descriptor encoding and kernel dispatch.
+// Every numeric step runs in the kernels; this file only checks and routes.
+#include <string.h>
+
+#include "dsa_kernels.h"
+
+using namespace dsa;
+
+namespace {
+
+constexpr size_t kHdr = 256;
+constexpr int64_t kTcIndexerMinRows = 64;  // prefill-shaped query sets use the tensor-core indexer
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_seqs(const dsa_seqs* s) {
+    if (!s || s->batch < 1 || !s->cu_seqlens_q || !s->cu_seqlens_k) return DSA_ERR_INVALID_ARG;
+    if (s->total_q < 0 || s->total_k < 0 || s->max_seqlen_q < 0 || s->max_seqlen_k < 0) return DSA_ERR_INVALID_ARG;
+    if (s->total_k >= (int64_t)1 << 31 || s->total_q >= (int64_t)1 << 31) return DSA_ERR_UNSUPPORTED;
+    if (s->max_seqlen_q > s->total_q || s->max_seqlen_k > s->total_k) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+int check_indexer(const dsa_seqs* s, const dsa_indexer_args* ia) {
+    if (!ia) return DSA_ERR_INVALID_ARG;
+    if (ia->dtype == DSA_F32) {
+        if (ia->w_dtype != DSA_F32 || ia->q_idx_scale || ia->k_idx_scale) return DSA_ERR_UNSUPPORTED;
+    } else if (ia->dtype == DSA_E4M3) {
+        if (ia->w_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+        if ((s->total_q && !ia->q_idx_scale) || (s->total_k && !ia->k_idx_scale)) return DSA_ERR_INVALID_ARG;
+    } else {
+        return DSA_ERR_UNSUPPORTED;
+    }
+    if (!ia->w_index || (s->total_q && !ia->q_idx) || (s->total_k && !ia->k_idx)) return DSA_ERR_INVALID_ARG;
+    if (!aligned(ia->q_idx, 16) || !aligned(ia->k_idx, 16) || !aligned(ia->w_index, 16)) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+bool attn_is_tc(const dsa_attn_args* aa) { return aa->dtype == DSA_BF16; }
+bool attn_v_separate(const dsa_attn_args* aa) { return !(aa->v == aa->k && aa->v_stride == aa->k_stride); }
+
+int check_attn(const dsa_seqs* s, const dsa_attn_args* aa) {
+    if (!aa) return DSA_ERR_INVALID_ARG;
+    if (s->total_q && (!aa->q || !aa->out)) return DSA_ERR_INVALID_ARG;
+    if (s->total_k && (!aa->k || !aa->v)) return DSA_ERR_INVALID_ARG;
+    if (aa->dtype == DSA_BF16) {
+        if (aa->heads != 128 || aa->dk != 576 || aa->dv != 512) return DSA_ERR_UNSUPPORTED;
+        if (!aligned(aa->q, 16) || !aligned(aa->k, 16) || !aligned(aa->v, 16) || !aligned(aa->out, 16))
+            return DSA_ERR_INVALID_ARG;
+        if (aa->k_stride < 576 || aa->v_stride < 512 || aa->k_stride % 8 || aa->v_stride % 8) return DSA_ERR_INVALID_ARG;
+        if (aa->q_stride_tok % 8 || aa->q_stride_head % 8 || aa->out_stride_tok % 8 || aa->out_stride_head % 8)
+            return DSA_ERR_INVALID_ARG;
+    } else if (aa->dtype == DSA_F32) {
+        if (aa->heads < 1 || aa->heads > 32) return DSA_ERR_UNSUPPORTED;
+        const bool okd = (aa->dk % 32 == 0 && aa->dk >= 32 && aa->dk <= 128);
+        const bool okv = (aa->dv % 32 == 0 && aa->dv >= 32 && aa->dv <= 128);
+        if (!okd || !okv) return DSA_ERR_UNSUPPORTED;
+        if (aa->k_stride < aa->dk || aa->v_stride < aa->dv) return DSA_ERR_INVALID_ARG;
+    } else {
+        return DSA_ERR_UNSUPPORTED;
+    }
+    if (aa->q_stride_head < aa->dk || aa->q_stride_tok < (int64_t)aa->heads * aa->q_stride_head) return DSA_ERR_INVALID_ARG;
+    if (aa->out_stride_head < aa->dv || aa->out_stride_tok < (int64_t)aa->heads * aa->out_stride_head)
+        return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+bool use_tc_indexer(const dsa_seqs* s, const dsa_indexer_args* ia) {
+    return ia->dtype == DSA_E4M3 && s->max_seqlen_q >= kTcIndexerMinRows;
+}
+
+struct WsLayout {
+    size_t u, s_row, idx, scores, total;
+};
+
+WsLayout ws_layout(const dsa_seqs* s, const dsa_indexer_args* ia, int32_t k, bool with_idx, bool with_scores) {
+    WsLayout L;
+    size_t off = kHdr;
+    const size_t ub = (ia && ia->dtype == DSA_F32) ? 4 : 1;
+    L.u = off;
+    off = align256(off + (size_t)s->total_q * 128 * ub);
+    L.s_row = off;
+    off = align256(off + (size_t)s->total_q * 4);
+    L.idx = off;
+    if (with_idx) off = align256(off + (size_t)s->total_q * (size_t)k * 4);
+    L.scores = off;
+    if (with_scores) off = align256(off + (size_t)s->total_q * (size_t)s->max_seqlen_k * 4);
+    L.total = off;
+    return L;
+}
+
+SeqView seq_view(const dsa_seqs* s) {
+    SeqView v;
+    v.batch = s->batch;
+    v.cu_q = s->cu_seqlens_q;
+    v.cu_k = s->cu_seqlens_k;
+    return v;
+}
+
+StatusHdr* hdr(void* ws) { return (StatusHdr*)ws; }
+
+int check_ws(void* ws, size_t have, size_t need) {
+    if (!ws || !aligned(ws, 256)) return DSA_ERR_INVALID_ARG;
+    if (have < need) return DSA_ERR_WORKSPACE;
+    return DSA_OK;
+}
+
+int cuda_status() { return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+// ---- TMA descriptors through the driver entry point (no link-time libcuda) ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiledFn) nullptr;
+        return (EncodeTiledFn)p;
+    }();
+    return fn;
+}
+
+// 2-D row-major map: `cols` x `rows` elements, row pitch in bytes, box
+// box_cols x box_rows, 128-byte swizzle.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t rows,
+                 uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int run_fold(const dsa_seqs* s, const dsa_indexer_args* ia, void* u, float* s_row, cudaStream_t st) {
+    FoldArgs f;
+    f.T = s->total_q;
+    f.idx_dtype = ia->dtype;
+    f.q_idx = ia->q_idx;
+    f.q_scale = ia->q_idx_scale;
+    f.w_dtype = ia->w_dtype;
+    f.W = ia->w_index;
+    f.u_out = u;
+    f.s_row_out = s_row;
+    launch_fold(f, st);
+    return cuda_status();
+}
+
+int run_scores_simt(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u, const float* s_row, int64_t row_begin,
+                    int64_t row_count, float* scores, int64_t ld, StatusHdr* h, cudaStream_t st) {
+    ScoresSimtArgs a;
+    a.sv = seq_view(s);
+    a.idx_dtype = ia->dtype;
+    a.u = u;
+    a.s_row = s_row;
+    a.k_idx = ia->k_idx;
+    a.k_scale = ia->k_idx_scale;
+    a.row_begin = row_begin;
+    a.row_count = row_count;
+    a.max_seqlen_k = s->max_seqlen_k;
+    a.scores = scores;
+    a.ld = ld;
+    a.st = h;
+    launch_scores_simt(a, st);
+    return cuda_status();
+}
+
+int run_indexer_tc(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u, const float* s_row, int mode, int32_t k,
+                   int32_t* idx, int64_t ld_idx, float* scores, int64_t ld_scores, int64_t row_begin, int64_t row_count,
+                   StatusHdr* h, cudaStream_t st) {
+    IndexerTcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.sv = seq_view(s);
+    a.mode = mode;
+    a.total_q = s->total_q;
+    a.max_seqlen_q = s->max_seqlen_q;
+    a.s_row = s_row;
+    a.k_scale = ia->k_idx_scale;
+    a.k = k;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.scores = scores;
+    a.ld_scores = ld_scores;
+    a.row_begin = row_begin;
+    a.row_count = row_count;
+    a.st = h;
+    if (!make_map_2d(&a.tm_u, CU_TENSOR_MAP_DATA_TYPE_UINT8, u, 128, (uint64_t)s->total_q, 128, 128, 128))
+        return DSA_ERR_CUDA;
+    if (!make_map_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, ia->k_idx, 128, (uint64_t)s->total_k, 128, 128, 256))
+        return DSA_ERR_CUDA;
+    if (!launch_indexer_tc(a, st)) return DSA_ERR_CUDA;
+    return cuda_status();
+}
+
+int run_topk(const dsa_seqs* s, const float* scores, int64_t ld, int64_t row_begin, int64_t row_count, int32_t k,
+             int32_t* idx, int64_t ld_idx, StatusHdr* h, cudaStream_t st) {
+    TopkArgs a;
+    a.sv = seq_view(s);
+    a.scores = scores;
+    a.ld = ld;
+    a.row_begin = row_begin;
+    a.row_count = row_count;
+    a.k = k;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.st = h;
+    launch_topk_rows(a, st);
+    return cuda_status();
+}
+
+int run_attn(const dsa_seqs* s, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel, StatusHdr* h,
+             cudaStream_t st) {
+    if (s->total_q == 0) return DSA_OK;
+    if (attn_is_tc(aa)) {
+        AttnTcArgs a;
+        memset(&a, 0, sizeof(a));
+        a.sv = seq_view(s);
+        a.total_q = s->total_q;
+        a.q = (const __nv_bfloat16*)aa->q;
+        a.q_stride_tok = aa->q_stride_tok;
+        a.q_stride_head = aa->q_stride_head;
+        a.scale_log2 = aa->scale * 1.4426950408889634f;
+        a.out = (__nv_bfloat16*)aa->out;
+        a.out_stride_tok = aa->out_stride_tok;
+        a.out_stride_head = aa->out_stride_head;
+        a.lse = aa->lse;
+        a.idx = idx;
+        a.ld_idx = ld_idx;
+        a.k_sel = k_sel;
+        a.v_separate = attn_v_separate(aa) ? 1 : 0;
+        a.st = h;
+        const uint64_t rows = (uint64_t)(s->total_k > 0 ? s->total_k : 1);
+        if (!make_map_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, aa->k, 576, rows, (uint64_t)aa->k_stride * 2, 64, 1))
+            return DSA_ERR_CUDA;
+        if (a.v_separate &&
+            !make_map_2d(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, aa->v, 512, rows, (uint64_t)aa->v_stride * 2, 64, 1))
+            return DSA_ERR_CUDA;
+        if (!launch_attn_tc(a, st)) return DSA_ERR_CUDA;
+        return cuda_status();
+    }
+    AttnF32Launch L;
+    L.sv = seq_view(s);
+    L.a.heads = aa->heads;
+    L.a.q = (const float*)aa->q;
+    L.a.q_stride_tok = aa->q_stride_tok;
+    L.a.q_stride_head = aa->q_stride_head;
+    L.a.k = (const float*)aa->k;
+    L.a.k_stride = aa->k_stride;
+    L.a.v = (const float*)aa->v;
+    L.a.v_stride = aa->v_stride;
+    L.a.scale = aa->scale;
+    L.a.out = (float*)aa->out;
+    L.a.out_stride_tok = aa->out_stride_tok;
+    L.a.out_stride_head = aa->out_stride_head;
+    L.a.lse = aa->lse;
+    L.dk = aa->dk;
+    L.dv = aa->dv;
+    L.total_q = s->total_q;
+    L.idx = idx;
+    L.ld_idx = ld_idx;
+    L.k_sel = k_sel;
+    L.st = h;
+    if (!launch_attn_f32(L, st)) return DSA_ERR_UNSUPPORTED;
+    return cuda_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_status_string(int status) {
+    switch (status) {
+        case DSA_OK: return "ok";
+        case DSA_ERR_INVALID_ARG: return "invalid argument";
+        case DSA_ERR_UNSUPPORTED: return "unsupported dtype/shape combination";
+        case DSA_ERR_WORKSPACE: return "workspace too small";
+        case DSA_ERR_CUDA: return "CUDA error";
+        case DSA_ERR_TIMEOUT: return "device wait timed out";
+        case DSA_ERR_INDEX: return "index or sequence bounds out of range";
+    }
+    return "unknown status";
+}
+
+int dsa_version(void) { return 1000; }
+
+int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexer_args* ia, const dsa_attn_args* aa,
+                       size_t* bytes) {
+    (void)aa;
+    if (!bytes) return DSA_ERR_INVALID_ARG;
+    int r = check_seqs(seqs);
+    if (r) return r;
+    switch (op) {
+        case DSA_OP_FOLD:
+        case DSA_OP_TOPK:
+        case DSA_OP_SPARSE_ATTN: *bytes = kHdr; return DSA_OK;
+        case DSA_OP_INDEX_SCORES:
+            if (!ia) return DSA_ERR_INVALID_ARG;
+            *bytes = ws_layout(seqs, ia, 0, false, false).total;
+            return DSA_OK;
+        case DSA_OP_FORWARD:
+            if (!ia || k < 1) return DSA_ERR_INVALID_ARG;
+            *bytes = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia)).total;
+            return DSA_OK;
+    }
+    return DSA_ERR_INVALID_ARG;
+}
+
+int dsa_fold(const dsa_seqs* seqs, const dsa_indexer_args* ia, void* u_out, float* s_row_out, void* ws, size_t ws_bytes,
+             dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_indexer(seqs, ia);
+    if (!r && seqs->total_q && (!u_out || !s_row_out)) r = DSA_ERR_INVALID_ARG;
+    if (!r) r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    return run_fold(seqs, ia, u_out, s_row_out, (cudaStream_t)stream);
+}
+
+int dsa_index_scores(const dsa_seqs* seqs, const dsa_indexer_args* ia, int64_t row_begin, int64_t row_count,
+                     float* scores, int64_t ld_scores, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_indexer(seqs, ia);
+    if (r) return r;
+    if (row_begin < 0 || row_count < 0 || row_begin + row_count > seqs->total_q) return DSA_ERR_INVALID_ARG;
+    if (row_count && (!scores || ld_scores < seqs->max_seqlen_k)) return DSA_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(seqs, ia, 0, false, false);
+    r = check_ws(ws, ws_bytes, L.total);
+    if (r) return r;
+    if (row_count == 0) return DSA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* w = (uint8_t*)ws;
+    r = run_fold(seqs, ia, w + L.u, (float*)(w + L.s_row), st);
+    if (r) return r;
+    if (use_tc_indexer(seqs, ia)) {
+        launch_fill_neg_inf(scores, row_count, ld_scores, st);
+        return run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 1, 0, nullptr, 0, scores, ld_scores,
+                              row_begin, row_count, hdr(ws), st);
+    }
+    return run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), row_begin, row_count, scores, ld_scores,
+                           hdr(ws), st);
+}
+
+int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_scores, int64_t row_begin, int64_t row_count,
+             int32_t k, int32_t* idx, int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (r) return r;
+    if (k < 1 || row_begin < 0 || row_count < 0 || row_begin + row_count > seqs->total_q) return DSA_ERR_INVALID_ARG;
+    if (row_count && (!scores || !idx || ld_scores < seqs->max_seqlen_k || ld_idx < k)) return DSA_ERR_INVALID_ARG;
+    r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    return run_topk(seqs, scores, ld_scores, row_begin, row_count, k, idx, ld_idx, hdr(ws), (cudaStream_t)stream);
+}
+
+int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel,
+                    void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_attn(seqs, aa);
+    if (r) return r;
+    if (k_sel < 0 || ld_idx < k_sel || (seqs->total_q && k_sel && !idx)) return DSA_ERR_INVALID_ARG;
+    r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    return run_attn(seqs, aa, idx, ld_idx, k_sel, hdr(ws), (cudaStream_t)stream);
+}
+
+int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k, int32_t* idx_out,
+                int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_indexer(seqs, ia);
+    if (!r) r = check_attn(seqs, aa);
+    if (r) return r;
+    if (k < 1) return DSA_ERR_INVALID_ARG;
+    if (idx_out && ld_idx < k) return DSA_ERR_INVALID_ARG;
+    const bool tc = use_tc_indexer(seqs, ia);
+    const WsLayout L = ws_layout(seqs, ia, k, true, !tc);
+    r = check_ws(ws, ws_bytes, L.total);
+    if (r) return r;
+    if (seqs->total_q == 0) return DSA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* w = (uint8_t*)ws;
+    int32_t* idx = idx_out ? idx_out : (int32_t*)(w + L.idx);
+    const int64_t ldi = idx_out ? ld_idx : k;
+    r = run_fold(seqs, ia, w + L.u, (float*)(w + L.s_row), st);
+    if (r) return r;
+    if (tc) {
+        r = run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, k, idx, ldi, nullptr, 0, 0, 0, hdr(ws), st);
+    } else {
+        float* sc = (float*)(w + L.scores);
+        const int64_t ld = seqs->max_seqlen_k;
+        r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st);
+        if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st);
+    }
+    if (r) return r;
+    return run_attn(seqs, aa, idx, ldi, k, hdr(ws), st);
+}
+
+int dsa_sync_status(void* ws, dsa_stream_t stream, int64_t* detail) {
+    if (!ws) return DSA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    StatusHdr h;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(h), st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (detail) *detail = h.detail;
+    return h.code;
+}
+
+int dsa_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t budget_cycles, dsa_stream_t stream) {
+    int r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    if (budget_cycles < 1 || budget_cycles > ((int64_t)1 << 34)) return DSA_ERR_INVALID_ARG;
+    launch_selftest_wait(hdr(ws), (long long)budget_cycles, (cudaStream_t)stream);
+    return cuda_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+// dsa_kernels.h -- internal launch interface between the C-ABI layer
+// (api.cu) and the kernel translation units.  Not part of the public ABI.
+#pragma once
+#include "dsa_device.cuh"
+
+namespace dsa {
+
+struct FoldArgs {
+    int64_t T;
+    int idx_dtype;
+    const void* q_idx;
+    const float* q_scale;
+    int w_dtype;
+    const void* W;
+    void* u_out;
+    float* s_row_out;
+};
+void launch_fold(const FoldArgs& a, cudaStream_t s);
+
+void launch_fill_neg_inf(float* p, int64_t rows, int64_t ld, cudaStream_t s);
+
+// Scores into memory with CUDA cores: fp32 indexer, or FP8 scan for short
+// query sets.  Entries s > pos are -inf.
+struct ScoresSimtArgs {
+    SeqView sv;
+    int idx_dtype;
+    const void* u;  // folded query [total_q,128] (f32 or e4m3 codes)
+    const float* s_row;
+    const void* k_idx;
+    const float* k_scale;
+    int64_t row_begin, row_count, max_seqlen_k;
+    float* scores;
+    int64_t ld;
+    StatusHdr* st;
+};
+void launch_scores_simt(const ScoresSimtArgs& a, cudaStream_t s);
+
+struct TopkArgs {
+    SeqView sv;
+    const float* scores;
+    int64_t ld, row_begin, row_count;
+    int k;
+    int32_t* idx;
+    int64_t ld_idx;
+    StatusHdr* st;
+};
+void launch_topk_rows(const TopkArgs& a, cudaStream_t s);
+
+struct AttnF32Args {
+    int heads;
+    const float* q;
+    int64_t q_stride_tok, q_stride_head;
+    const float* k;
+    int64_t k_stride;
+    const float* v;
+    int64_t v_stride;
+    float scale;
+    float* out;
+    int64_t out_stride_tok, out_stride_head;
+    float* lse;
+};
+struct AttnF32Launch {
+    SeqView sv;
+    AttnF32Args a;
+    int dk, dv;
+    int64_t total_q;
+    const int32_t* idx;
+    int64_t ld_idx;
+    int k_sel;
+    StatusHdr* st;
+};
+bool launch_attn_f32(const AttnF32Launch& L, cudaStream_t s);
+
+void launch_selftest_wait(StatusHdr* st, long long budget, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// tcgen05 FP8 lightning indexer with the fused exact top-k (prefill shapes).
+// mode 0: fused selection -> idx; mode 1: write scores (rows in range).
+// ---------------------------------------------------------------------------
+struct IndexerTcArgs {
+    SeqView sv;
+    int mode;
+    int64_t total_q, max_seqlen_q;
+    const float* s_row;     // [total_q]
+    const float* k_scale;   // [total_k]
+    int k;                  // top-k size (mode 0)
+    int32_t* idx;           // mode 0: [total_q, ld_idx]
+    int64_t ld_idx;
+    float* scores;          // mode 1: [row_count, ld]
+    int64_t ld_scores, row_begin, row_count;
+    StatusHdr* st;
+    CUtensorMap tm_u;       // folded query codes [total_q,128], box 128x128
+    CUtensorMap tm_k;       // key codes [total_k,128], box 128x256
+};
+bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s);
+extern const int kIndexerRowsPerBlock;
+
+// ---------------------------------------------------------------------------
+// tcgen05 BF16 sparse MQA attention, 128 heads, dk 576, dv 512, CTA pairs.
+// ---------------------------------------------------------------------------
+struct AttnTcArgs {
+    SeqView sv;
+    int64_t total_q;
+    const __nv_bfloat16* q;
+    int64_t q_stride_tok, q_stride_head;
+    float scale_log2;       // softmax scale * log2(e)
+    __nv_bfloat16* out;
+    int64_t out_stride_tok, out_stride_head;
+    float* lse;
+    const int32_t* idx;
+    int64_t ld_idx;
+    int k_sel;
+    int v_separate;         // 0: V = K[:, :512] (same rows); 1: own tensor
+    StatusHdr* st;
+    CUtensorMap tm_k;       // K rows [total_k, 576], box 64x1, 128B swizzle
+    CUtensorMap tm_v;       // V rows [total_k, 512] (v_separate)
+};
+bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s);
+
+}  // namespace dsa

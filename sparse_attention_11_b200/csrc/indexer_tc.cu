@@ -1,0 +1,351 @@
+// indexer_tc.cu -- lightning indexer on the 5th-generation tensor cores with
+// the exact per-query top-k fused onto the score tiles.
+//
+// Method: "DeepSeek-V3.2与稀疏注意力技术革新", §2.2 (I[t,s] = ReLU(q_t W k_s)
+// with 128-dim FP8 keys; W is folded into the query beforehand) and §2.3
+// (each query keeps its k best keys; the page maintains the candidates with
+// a "dynamic priority queue" -- here the exact selection is reached by a
+// most-significant-digit radix descent over repeated score sweeps, so the
+// L x L score matrix never leaves the SM).
+//
+// Work unit: a block of 128 consecutive queries of one sequence.  One CTA
+// per block, 6 warps:
+//   warp 0      TMA producer: the block's folded queries (128 x 128 e4m3,
+//               once) and key tiles of 256 x 128 e4m3 (+ their fp32 scales)
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f8f6f4,
+//               M=128 N=256 K=32, fp32 accumulators in two TMEM buffers
+//   warps 2..5  epilogue: thread <-> query row (its TMEM lane); reads a
+//               row of 256 fp32 dots per tile, forms the score
+//               ReLU((dot * s_k) * s_row) and applies the sweep's action.
+//
+// Sweeps over the block's causal key tiles (a block stops as soon as every
+// row's selection is determined):
+//   HIST level 1..4  per-row histogram of the next radix digit of the score
+//                    bits, over the keys of the row's current bucket
+//   EMIT             writes each row's selected indices in ascending order
+// Score keys are the fp32 bit patterns (non-negative after ReLU).  Digit
+// 1 is ceil(bits / 2^23) (0 only for +0.0), then bits 22..15, 14..7, 6..0 of
+// (bits - 1).  After each histogram the row knows how many keys lie above
+// the bucket holding its K-th best; it stops refining once that bucket is
+// taken whole or holds a single value (ties: lowest indices first, which
+// the ascending emission order gives for free).
+#include "dsa_kernels.h"
+
+namespace dsa {
+
+constexpr int IX_BM = 128;
+constexpr int IX_BN = 256;
+constexpr int IX_NST = 2;
+const int kIndexerRowsPerBlock = IX_BM;
+
+constexpr uint32_t IX_A_BYTES = IX_BM * 128;
+constexpr uint32_t IX_B_BYTES = IX_BN * 128;
+constexpr uint32_t IX_OFF_A = 0;
+constexpr uint32_t IX_OFF_B = IX_OFF_A + IX_A_BYTES;
+constexpr uint32_t IX_OFF_SC = IX_OFF_B + IX_NST * IX_B_BYTES;
+constexpr uint32_t IX_OFF_HIST = IX_OFF_SC + IX_NST * IX_BN * 4;
+constexpr uint32_t IX_OFF_BAR = IX_OFF_HIST + 256 * IX_BM * 4;
+constexpr uint32_t IX_SMEM = IX_OFF_BAR + 256 + 1024;  // + alignment slack
+
+enum : int { SW_STOP = 0, SW_HIST = 1, SW_EMIT = 2, SW_SCORES = 3 };
+
+struct IxBars {
+    uint64_t full[IX_NST];
+    uint64_t empty[IX_NST];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t a_full;
+    uint64_t dec;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int next_kind;
+    int next_level;
+    int any_unresolved;
+    int abort;
+};
+
+__global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constant__ IndexerTcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    IxBars* bars = (IxBars*)(smem + IX_OFF_BAR);
+    float* sc_s = (float*)(smem + IX_OFF_SC);
+    uint32_t* hist = (uint32_t*)(smem + IX_OFF_HIST);
+    const uint32_t warp = warp_id(), lane = lane_id();
+    StatusHdr* st = a.st;
+    volatile int* abort = &bars->abort;
+
+    // ---- block -> (sequence, row range); heaviest blocks launch first ----
+    const int64_t nblk = (a.max_seqlen_q + IX_BM - 1) / IX_BM;
+    const int b = (int)(blockIdx.x % a.sv.batch);
+    const int64_t jb = nblk - 1 - (int64_t)(blockIdx.x / a.sv.batch);
+    const int64_t q0 = __ldg(a.sv.cu_q + b), sq = __ldg(a.sv.cu_q + b + 1) - q0;
+    const int64_t key_base = __ldg(a.sv.cu_k + b), sk = __ldg(a.sv.cu_k + b + 1) - key_base;
+    const int64_t i0 = jb * IX_BM;
+    if (i0 >= sq) return;
+    const int64_t nrows = min((int64_t)IX_BM, sq - i0);
+    const int64_t pos_first = sk - sq + i0;
+    const int64_t pos_last = pos_first + nrows - 1;
+    if (pos_first < 0) {
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, q0 + i0);
+        return;
+    }
+    const int64_t t_first = q0 + i0;
+    if (a.mode == 1 && (t_first + nrows <= a.row_begin || t_first >= a.row_begin + a.row_count)) return;
+    const int n_tiles = (int)((pos_last + IX_BN) / IX_BN);
+    int first_kind;
+    if (a.mode == 1)
+        first_kind = SW_SCORES;
+    else
+        first_kind = (pos_last + 1 > a.k) ? SW_HIST : SW_STOP;
+
+    const uint32_t sA = smem_u32(smem + IX_OFF_A);
+    const uint32_t sB = smem_u32(smem + IX_OFF_B);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < IX_NST; ++i) {
+            mbar_init(smem_u32(&bars->full[i]), 1);
+            mbar_init(smem_u32(&bars->empty[i]), 1 + 4);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bars->acc_full[i]), 1);
+            mbar_init(smem_u32(&bars->acc_empty[i]), 4);
+        }
+        mbar_init(smem_u32(&bars->a_full), 1);
+        mbar_init(smem_u32(&bars->dec), 1);
+        mbar_init(smem_u32(&bars->drain), 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            tma_prefetch_desc(&a.tm_u);
+            tma_prefetch_desc(&a.tm_k);
+        }
+        if (first_kind != SW_STOP) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(smem_u32(&bars->a_full), IX_A_BYTES);
+                tma_load_2d(sA, &a.tm_u, 0, (int32_t)t_first, smem_u32(&bars->a_full));
+            }
+            uint32_t g = 0;
+            uint32_t last_issued[IX_NST];
+            for (int i = 0; i < IX_NST; ++i) last_issued[i] = 0xFFFFFFFFu;
+            int kind = first_kind;
+            for (int sw = 0; kind != SW_STOP; ++sw) {
+                for (int tile = 0; tile < n_tiles; ++tile, ++g) {
+                    const uint32_t s = g % IX_NST;
+                    if (!wait_warp(smem_u32(&bars->empty[s]), ((g / IX_NST) & 1) ^ 1, abort, st, 0x1101)) break;
+                    const int64_t kr0 = key_base + (int64_t)tile * IX_BN;
+                    float* scs = sc_s + s * IX_BN;
+                    for (int i = lane; i < IX_BN; i += 32) {
+                        const int64_t kr = kr0 + i;
+                        scs[i] = (tile * IX_BN + i <= pos_last) ? __ldg(a.k_scale + kr) : 0.f;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(smem_u32(&bars->full[s]), IX_B_BYTES);
+                        tma_load_2d(sB + s * IX_B_BYTES, &a.tm_k, 0, (int32_t)kr0, smem_u32(&bars->full[s]));
+                    }
+                    last_issued[s] = g;
+                    __syncwarp();
+                }
+                if (*abort) break;
+                if (!wait_warp(smem_u32(&bars->dec), sw & 1, abort, st, 0x1102)) break;
+                kind = *(volatile int*)&bars->next_kind;
+            }
+            // drain: every issued load must land before the CTA exits
+            if (*abort && lane == 0) {
+                for (int s = 0; s < IX_NST; ++s)
+                    if (last_issued[s] != 0xFFFFFFFFu)
+                        mbar_wait(smem_u32(&bars->full[s]), (last_issued[s] / IX_NST) & 1, nullptr, st, 0x1103, 1ll << 28);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        constexpr uint32_t idesc = idesc_make(0, 0, false, IX_BM, IX_BN);
+        if (first_kind != SW_STOP) {
+            bool ok = wait_warp(smem_u32(&bars->a_full), 0, abort, st, 0x1201);
+            uint32_t g = 0;
+            int kind = first_kind;
+            for (int sw = 0; ok && kind != SW_STOP; ++sw) {
+                for (int tile = 0; tile < n_tiles; ++tile, ++g) {
+                    const uint32_t s = g % IX_NST, ab = g & 1;
+                    if (!wait_warp(smem_u32(&bars->full[s]), (g / IX_NST) & 1, abort, st, 0x1202)) { ok = false; break; }
+                    if (!wait_warp(smem_u32(&bars->acc_empty[ab]), ((g >> 1) & 1) ^ 1, abort, st, 0x1203)) { ok = false; break; }
+                    tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad = sdesc_sw128(sA + ks * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(sB + s * IX_B_BYTES + ks * 32, 16, 1024);
+                            mma_fp8_ss(tmem + ab * IX_BN, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit(smem_u32(&bars->empty[s]));
+                        mma_commit(smem_u32(&bars->acc_full[ab]));
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (!wait_warp(smem_u32(&bars->dec), sw & 1, abort, st, 0x1204)) break;
+                kind = *(volatile int*)&bars->next_kind;
+            }
+            if (*abort && lane == 0) {
+                mma_commit(smem_u32(&bars->drain));
+                mbar_wait(smem_u32(&bars->drain), 0, nullptr, st, 0x1205, 1ll << 28);
+            }
+        }
+    } else {
+        // ================= epilogue: thread <-> query row =================
+        const uint32_t quad = warp & 3;
+        const int row = (int)(quad * 32 + lane);
+        const bool has_row = row < nrows;
+        const int64_t t = t_first + row;
+        const int64_t pos = pos_first + row;
+        const float srow = has_row ? __ldg(a.s_row + t) : 0.f;
+        const bool in_range = a.mode != 1 || (t >= a.row_begin && t < a.row_begin + a.row_count);
+        const bool take_all = pos + 1 <= a.k;
+        // radix state
+        int level = 0, sh = 31, P = 0;
+        uint32_t need = (uint32_t)a.k;
+        bool resolved = !has_row || take_all;
+        uint32_t* myhist = hist + row;  // bin b at myhist[b * IX_BM]
+        int32_t* out = (a.mode == 0 && has_row) ? a.idx + t * a.ld_idx : nullptr;
+        float* srow_out = (a.mode == 1 && has_row && in_range) ? a.scores + (t - a.row_begin) * a.ld_scores : nullptr;
+        int cnt = 0;
+        uint32_t taken = 0;
+        for (int i = 0; i < 256; ++i) myhist[i * IX_BM] = 0;
+
+        uint32_t g = 0;
+        int kind = first_kind;
+        for (int sw = 0; kind != SW_STOP; ++sw) {
+            const int lvl = level + 1;  // histogram level of this sweep (HIST)
+            for (int tile = 0; tile < n_tiles; ++tile, ++g) {
+                const uint32_t s = g % IX_NST, ab = g & 1;
+                bool ok = wait_warp(smem_u32(&bars->acc_full[ab]), (g >> 1) & 1, abort, st, 0x1301);
+                ok = ok && wait_warp(smem_u32(&bars->full[s]), (g / IX_NST) & 1, abort, st, 0x1302);
+                tc_fence_after();
+                const float* scs = sc_s + s * IX_BN;
+                const int64_t s_tile = (int64_t)tile * IX_BN;
+                const bool active = ok && has_row && !(kind == SW_HIST && resolved);
+#pragma unroll 1
+                for (int ch = 0; ch < IX_BN / 32; ++ch) {
+                    uint32_t v[32];
+                    if (ok) {
+                        tmem_ld32(tmem + ((quad * 32) << 16) + ab * IX_BN + ch * 32, v);
+                        tmem_wait_ld();
+                    }
+                    if (!active) continue;
+                    const int64_t sbase = s_tile + ch * 32;
+                    if (sbase > pos) continue;
+                    const int lim = (int)min((int64_t)31, pos - sbase);  // columns 0..lim are causal
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (i > lim) break;
+                        const float x = __fmul_rn(__fmul_rn(__uint_as_float(v[i]), scs[ch * 32 + i]), srow);
+                        int kb = max(__float_as_int(x), 0);
+                        kb = min(kb, 0x7F800000);
+                        const int32_t sidx = (int32_t)(sbase + i);
+                        if (kind == SW_HIST) {
+                            if (lvl == 1) {
+                                atomicAdd(&myhist[((uint32_t)kb + 0x7FFFFFu) >> 23 << 7], 1u);
+                            } else {
+                                const int xk = kb - 1;
+                                if ((xk >> sh) == P) {
+                                    const uint32_t d = lvl == 2 ? ((uint32_t)xk >> 15) & 255u
+                                                     : lvl == 3 ? ((uint32_t)xk >> 7) & 255u
+                                                                : (uint32_t)xk & 127u;
+                                    atomicAdd(&myhist[d << 7], 1u);
+                                }
+                            }
+                        } else if (kind == SW_EMIT) {
+                            bool e = take_all;
+                            if (!e) {
+                                const int hi = (kb - 1) >> sh;
+                                if (hi > P) e = true;
+                                else if (hi == P && taken < need) { e = true; ++taken; }
+                            }
+                            if (e) {
+                                if (cnt < a.k) out[cnt] = sidx;
+                                ++cnt;
+                            }
+                        } else if (kind == SW_SCORES) {
+                            if (srow_out) srow_out[sidx] = __int_as_float(kb);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&bars->acc_empty[ab]));
+                    mbar_arrive(smem_u32(&bars->empty[s]));
+                }
+            }
+            // ---- end of sweep: refine each row's bucket; one thread decides ----
+            if (kind == SW_HIST) {
+                if (has_row && !resolved) {
+                    uint32_t cum = 0;
+                    int bsel = 0;
+                    const int top = lvl == 4 ? 127 : 255;
+                    for (int bb = top; bb >= 0; --bb) {
+                        const uint32_t c = myhist[bb * IX_BM];
+                        if (cum + c >= need) { bsel = bb; break; }
+                        cum += c;
+                    }
+                    const uint32_t in_bin = myhist[bsel * IX_BM];
+                    need -= cum;
+                    if (lvl == 1) { P = bsel - 1; sh = 23; }
+                    else if (lvl == 2) { P = (P << 8) | bsel; sh = 15; }
+                    else if (lvl == 3) { P = (P << 8) | bsel; sh = 7; }
+                    else { P = (P << 7) | bsel; sh = 0; }
+                    resolved = in_bin == need || P == -1 || lvl == 4;
+                }
+                level = lvl;
+                for (int i = 0; i < 256; ++i) myhist[i * IX_BM] = 0;
+                if (threadIdx.x == 64) bars->any_unresolved = 0;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (has_row && !resolved) bars->any_unresolved = 1;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (threadIdx.x == 64) {
+                int nk = kind == SW_HIST ? (bars->any_unresolved ? SW_HIST : SW_EMIT) : SW_STOP;
+                if (*abort) nk = SW_STOP;
+                bars->next_kind = nk;
+                mbar_arrive(smem_u32(&bars->dec));
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            kind = *(volatile int*)&bars->next_kind;
+        }
+        // ---- finish the index rows ----
+        if (a.mode == 0 && has_row) {
+            if (first_kind == SW_STOP) {  // every row of the block keeps its whole prefix
+                for (int64_t s = 0; s <= pos; ++s) out[s] = (int32_t)s;
+                cnt = (int)(pos + 1);
+            }
+            const int expect = (int)min((int64_t)a.k, pos + 1);
+            if (cnt != expect && !*abort) report(st, DSA_ERR_INDEX, -2000000 - t);
+            for (int s = min(cnt, a.k); s < a.k; ++s) out[s] = -1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s) {
+    if (cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM) != cudaSuccess)
+        return false;
+    const int64_t nblk = (a.max_seqlen_q + IX_BM - 1) / IX_BM;
+    const int64_t grid = nblk * a.sv.batch;
+    if (grid <= 0) return true;
+    indexer_tc_kernel<<<(unsigned)grid, 192, IX_SMEM, s>>>(a);
+    return cudaGetLastError() == cudaSuccess;
+}
+
+}  // namespace dsa

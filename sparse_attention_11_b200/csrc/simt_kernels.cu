@@ -1,0 +1,433 @@
+// simt_kernels.cu -- CUDA-core kernels of the DSA path:
+//   * fold of W_index into the indexer query (+ e4m3 requantisation)
+//   * fp32 indexer scores (tiny fp32 configuration)
+//   * FP8 indexer scan for short query sets (decode), HBM-bound
+//   * exact per-row radix top-k over scores held in memory
+//   * exact fp32 sparse attention (tiny fp32 configuration)
+//
+// Method: "DeepSeek-V3.2与稀疏注意力技术革新", §2.2 (indexer), §2.3 (top-k
+// selection, attention on the selected subset), §3.1 (MQA: heads share KV).
+#include <cuda_fp8.h>
+
+#include "dsa_device.cuh"
+#include "dsa_kernels.h"
+
+namespace dsa {
+
+// ---------------------------------------------------------------------------
+// a1: fold.  Thread j of a 128-thread CTA keeps column j of W in registers
+// and folds FOLD_ROWS query rows: u_j = sum_i q_i W[i][j] (fp32 FMA chain).
+// E4M3: s_u = amax/448 (IEEE division), codes = e4m3_rn_satfinite(u_j / s_u),
+// s_row = s_q * s_u.
+// ---------------------------------------------------------------------------
+constexpr int FOLD_ROWS = 32;
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+__global__ void __launch_bounds__(128) fold_kernel(int64_t T, int idx_dtype, const void* __restrict__ q_idx,
+                                                   const float* __restrict__ q_scale, int w_dtype,
+                                                   const void* __restrict__ W, void* __restrict__ u_out,
+                                                   float* __restrict__ s_row_out) {
+    __shared__ float qs[128];
+    __shared__ float red[4];
+    const int j = threadIdx.x;
+    float w[128];
+#pragma unroll
+    for (int i = 0; i < 128; ++i) {
+        if (w_dtype == DSA_F32)
+            w[i] = __ldg((const float*)W + i * 128 + j);
+        else
+            w[i] = __bfloat162float(((const __nv_bfloat16*)W)[i * 128 + j]);
+    }
+    const int64_t r0 = (int64_t)blockIdx.x * FOLD_ROWS;
+    for (int rr = 0; rr < FOLD_ROWS; ++rr) {
+        const int64_t r = r0 + rr;
+        if (r >= T) break;
+        __syncthreads();
+        if (idx_dtype == DSA_F32)
+            qs[j] = __ldg((const float*)q_idx + r * 128 + j);
+        else
+            qs[j] = e4m3_to_f32(((const uint8_t*)q_idx)[r * 128 + j]);
+        __syncthreads();
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc = fmaf(qs[i], w[i], acc);
+        if (idx_dtype == DSA_F32) {
+            ((float*)u_out)[r * 128 + j] = acc;
+            if (j == 0) s_row_out[r] = 1.0f;
+            continue;
+        }
+        float a = fabsf(acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if ((j & 31) == 0) red[j >> 5] = a;
+        __syncthreads();
+        const float amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        const float s_u = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+        const float y = amax == 0.f ? 0.f : __fdiv_rn(acc, s_u);
+        ((uint8_t*)u_out)[r * 128 + j] = (uint8_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+        if (j == 0) s_row_out[r] = __fmul_rn(__ldg(q_scale + r), s_u);
+    }
+}
+
+void launch_fold(const FoldArgs& a, cudaStream_t s) {
+    const int64_t grid = (a.T + FOLD_ROWS - 1) / FOLD_ROWS;
+    if (grid == 0) return;
+    fold_kernel<<<(unsigned)grid, 128, 0, s>>>(a.T, a.idx_dtype, a.q_idx, a.q_scale, a.w_dtype, a.W, a.u_out, a.s_row_out);
+}
+
+// ---------------------------------------------------------------------------
+// Fill a [rows, ld] float array with -inf.
+// ---------------------------------------------------------------------------
+__global__ void fill_neg_inf_kernel(float* p, int64_t rows, int64_t ld) {
+    const int64_t n = rows * ld;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = -INFINITY;
+}
+
+void launch_fill_neg_inf(float* p, int64_t rows, int64_t ld, cudaStream_t s) {
+    const int64_t n = rows * ld;
+    if (n <= 0) return;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    fill_neg_inf_kernel<<<(unsigned)blocks, 256, 0, s>>>(p, rows, ld);
+}
+
+// ReLU applied on the bit pattern: every x <= 0 (and -0.0) becomes +0.0;
+// +inf/NaN are clamped to +inf so that the key stays a finite-order value.
+__device__ __forceinline__ float relu_key(float x) {
+    int b = __float_as_int(x);
+    b = max(b, 0);
+    b = min(b, 0x7F800000);
+    return __int_as_float(b);
+}
+
+// ---------------------------------------------------------------------------
+// a2, fp32: scores[r, s] = ReLU(u_t . k_s) for s <= pos; grid (key chunks,
+// rows), one thread per key.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) scores_f32_kernel(SeqView sv, const float* __restrict__ u,
+                                                         const float* __restrict__ k_idx, int64_t row_begin,
+                                                         float* __restrict__ scores, int64_t ld, StatusHdr* st) {
+    __shared__ float us[128];
+    const int64_t r = blockIdx.y;
+    const int64_t t = row_begin + r;
+    const RowInfo ri = row_info(sv, t);
+    if (!ri.ok) {
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, t);
+        return;
+    }
+    us[threadIdx.x] = u[t * 128 + threadIdx.x];
+    __syncthreads();
+    const int64_t s = (int64_t)blockIdx.x * 128 + threadIdx.x;
+    if (s > ri.pos) return;
+    const float* kr = k_idx + (ri.key_base + s) * 128;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < 128; ++i) acc = fmaf(us[i], __ldg(kr + i), acc);
+    scores[r * ld + s] = relu_key(acc);
+}
+
+// ---------------------------------------------------------------------------
+// a2, FP8 scan for short query sets: 8 lanes per key (16 codes each), fp32
+// FMA of the exact e4m3 products, xor-shuffle reduction; score =
+// ReLU((dot * s_k) * s_row).  HBM-bound: 132 bytes read per key.
+// ---------------------------------------------------------------------------
+constexpr int SCAN_KEYS = 1024;
+
+__global__ void __launch_bounds__(256) scan_fp8_kernel(SeqView sv, const uint8_t* __restrict__ u8,
+                                                       const float* __restrict__ s_row, const uint8_t* __restrict__ k8,
+                                                       const float* __restrict__ k_scale, int64_t row_begin,
+                                                       float* __restrict__ scores, int64_t ld, StatusHdr* st) {
+    const int64_t r = blockIdx.y;
+    const int64_t t = row_begin + r;
+    const RowInfo ri = row_info(sv, t);
+    if (!ri.ok) {
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, t);
+        return;
+    }
+    const int sub = threadIdx.x & 7;  // which 16-byte slice of the key
+    float uq[16];
+    {
+        const uint4 v = *(const uint4*)(u8 + t * 128 + sub * 16);
+        const uint8_t* b = (const uint8_t*)&v;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) uq[i] = e4m3_to_f32(b[i]);
+    }
+    const float srow = s_row[t];
+    const int64_t s_begin = (int64_t)blockIdx.x * SCAN_KEYS;
+    const int64_t s_end = min(s_begin + SCAN_KEYS, ri.pos + 1);
+    for (int64_t s0 = s_begin; s0 < s_end; s0 += 32) {
+        const int64_t s = s0 + (threadIdx.x >> 3);
+        float acc = 0.f;
+        if (s < s_end) {
+            const uint4 v = __ldg((const uint4*)(k8 + (ri.key_base + s) * 128 + sub * 16));
+            const uint8_t* b = (const uint8_t*)&v;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc = fmaf(uq[i], e4m3_to_f32(b[i]), acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        if (sub == 0 && s < s_end) {
+            const float x = __fmul_rn(__fmul_rn(acc, __ldg(k_scale + ri.key_base + s)), srow);
+            scores[r * ld + s] = relu_key(x);
+        }
+    }
+}
+
+void launch_scores_simt(const ScoresSimtArgs& a, cudaStream_t s) {
+    if (a.row_count <= 0) return;
+    launch_fill_neg_inf(a.scores, a.row_count, a.ld, s);
+    if (a.idx_dtype == DSA_F32) {
+        dim3 grid((unsigned)((a.max_seqlen_k + 127) / 128), (unsigned)a.row_count);
+        scores_f32_kernel<<<grid, 128, 0, s>>>(a.sv, (const float*)a.u, (const float*)a.k_idx, a.row_begin, a.scores,
+                                                a.ld, a.st);
+    } else {
+        dim3 grid((unsigned)((a.max_seqlen_k + SCAN_KEYS - 1) / SCAN_KEYS), (unsigned)a.row_count);
+        scan_fp8_kernel<<<grid, 256, 0, s>>>(a.sv, (const uint8_t*)a.u, a.s_row, (const uint8_t*)a.k_idx, a.k_scale,
+                                             a.row_begin, a.scores, a.ld, a.st);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// a3: exact top-k of one row per CTA by most-significant-digit radix select
+// (4 digits of 8 bits over an order-preserving 32-bit key), then an
+// emission pass in ascending index order.  Ties at the threshold go to the
+// lowest indices.  Key order: NaN < -inf < ... < -0.0 == +0.0 < ... < +inf.
+// ---------------------------------------------------------------------------
+constexpr int TOPK_NT = 1024;
+
+__device__ __forceinline__ uint32_t order_key(float x) {
+    uint32_t u = __float_as_uint(x);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;  // NaN: below everything
+    if (u == 0x80000000u) u = 0u;                     // -0.0 == +0.0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix count of `flag` over the CTA (all TOPK_NT threads call).
+__device__ __forceinline__ int cta_excl_scan(int flag, int* warp_tot, int* total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const unsigned bal = __ballot_sync(0xffffffffu, flag);
+    const int in_warp = __popc(bal & ((1u << lane) - 1u));
+    __syncthreads();
+    if (lane == 0) warp_tot[w] = __popc(bal);
+    __syncthreads();
+    if (w == 0) {
+        int v = warp_tot[lane];
+        int inc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += n;
+        }
+        warp_tot[lane] = inc - v;
+        if (lane == 31) warp_tot[32] = inc;
+    }
+    __syncthreads();
+    *total = warp_tot[32];
+    return warp_tot[w] + in_warp;
+}
+
+__global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld,
+                                                            int64_t row_begin, int k, int32_t* __restrict__ idx,
+                                                            int64_t ld_idx, StatusHdr* st) {
+    __shared__ uint32_t hist[256];
+    __shared__ int warp_tot[33];
+    __shared__ uint32_t sel_bin, sel_above;
+    const int64_t r = blockIdx.x;
+    const int64_t t = row_begin + r;
+    const RowInfo ri = row_info(sv, t);
+    int32_t* out = idx + r * ld_idx;
+    if (!ri.ok) {
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, t);
+        return;
+    }
+    const int64_t n = ri.pos + 1;
+    const float* row = scores + r * ld;
+    if (n <= k) {
+        for (int64_t s = threadIdx.x; s < k; s += TOPK_NT) out[s] = s < n ? (int32_t)s : -1;
+        return;
+    }
+    uint32_t prefix = 0, mask = 0;
+    uint32_t need = (uint32_t)k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = threadIdx.x; i < 256; i += TOPK_NT) hist[i] = 0;
+        __syncthreads();
+        for (int64_t s = threadIdx.x; s < n; s += TOPK_NT) {
+            const uint32_t key = order_key(row[s]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            // lane l owns bins [8l, 8l+8); count above from the top
+            const int lane = threadIdx.x;
+            uint32_t c[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = hist[lane * 8 + i];
+                sum += c[i];
+            }
+            uint32_t above = 0;  // count in lanes > lane
+            uint32_t inc = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t v = __shfl_down_sync(0xffffffffu, inc, o);
+                if (lane + o < 32) inc += v;
+            }
+            above = inc - sum;
+            // the lane where the running count (from the top) first reaches need
+            const bool mine = above < need && above + sum >= need;
+            if (mine) {
+                uint32_t acc = above;
+                for (int i = 7; i >= 0; --i) {
+                    if (acc + c[i] >= need) {
+                        sel_bin = (uint32_t)(lane * 8 + i);
+                        sel_above = acc;
+                        break;
+                    }
+                    acc += c[i];
+                }
+            }
+        }
+        __syncthreads();
+        const uint32_t bin = sel_bin;
+        prefix |= bin << shift;
+        mask |= 0xFFu << shift;
+        need -= sel_above;
+        const uint32_t in_bin = hist[bin];
+        __syncthreads();
+        if (in_bin == need) break;
+    }
+    // emission in ascending index order
+    int base_out = 0, taken = 0;
+    for (int64_t s0 = 0; s0 < n; s0 += TOPK_NT) {
+        const int64_t s = s0 + threadIdx.x;
+        int above = 0, eq = 0;
+        if (s < n) {
+            const uint32_t m = order_key(row[s]) & mask;
+            above = m > prefix;
+            eq = m == prefix;
+        }
+        int eq_total;
+        const int eq_rank = cta_excl_scan(eq, warp_tot, &eq_total);
+        const int take = above || (eq && taken + eq_rank < (int)need);
+        int take_total;
+        const int at = cta_excl_scan(take, warp_tot, &take_total);
+        if (take) out[base_out + at] = (int32_t)s;
+        base_out += take_total;
+        taken += min(eq_total, max((int)need - taken, 0));
+    }
+    for (int64_t s = base_out + threadIdx.x; s < k; s += TOPK_NT) out[s] = -1;
+    if (threadIdx.x == 0 && base_out != k) report(st, DSA_ERR_INDEX, -1000000 - t);
+}
+
+void launch_topk_rows(const TopkArgs& a, cudaStream_t s) {
+    if (a.row_count <= 0) return;
+    topk_rows_kernel<<<(unsigned)a.row_count, TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k, a.idx, a.ld_idx,
+                                                              a.st);
+}
+
+// ---------------------------------------------------------------------------
+// a4, fp32: one warp per (query, head); online softmax over the selected
+// rows with expf; dk, dv <= 128 (multiples of 32).
+// ---------------------------------------------------------------------------
+template <int DK, int DV>
+__global__ void attn_f32_kernel(SeqView sv, AttnF32Args a, const int32_t* __restrict__ idx, int64_t ld_idx, int k_sel,
+                                StatusHdr* st) {
+    const int64_t t = blockIdx.x;
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (h >= a.heads) return;
+    const RowInfo ri = row_info(sv, t);
+    if (!ri.ok) {
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, t);
+        return;
+    }
+    constexpr int NQ = DK / 32, NV = DV / 32;
+    const float* qp = a.q + t * a.q_stride_tok + h * a.q_stride_head;
+    float q[NQ], o[NV];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) q[i] = qp[lane + 32 * i];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) o[i] = 0.f;
+    float m = -INFINITY, l = 0.f;
+    const int32_t* ir = idx + t * ld_idx;
+    for (int j = 0; j < k_sel; ++j) {
+        const int32_t v = ir[j];
+        if (v < 0) continue;
+        if (v >= ri.seqlen_k) {
+            if (lane == 0 && h == 0) report(st, DSA_ERR_INDEX, t);
+            continue;
+        }
+        const int64_t row = ri.key_base + v;
+        const float* kr = a.k + row * a.k_stride;
+        float d = 0.f;
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) d = fmaf(q[i], kr[lane + 32 * i], d);
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
+        const float z = d * a.scale;
+        if (z > m) {
+            const float c = expf(m - z);
+            l *= c;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) o[i] *= c;
+            m = z;
+        }
+        const float p = expf(z - m);
+        l += p;
+        const float* vr = a.v + row * a.v_stride;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) o[i] = fmaf(p, vr[lane + 32 * i], o[i]);
+    }
+    float* op = a.out + t * a.out_stride_tok + h * a.out_stride_head;
+    const float inv = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) op[lane + 32 * i] = o[i] * inv;
+    if (a.lse && lane == 0) a.lse[t * a.heads + h] = l > 0.f ? m + logf(l) : -INFINITY;
+}
+
+template <int DK>
+static bool launch_attn_f32_dk(int dv, const AttnF32Launch& L, cudaStream_t s) {
+    dim3 grid((unsigned)L.total_q), block((unsigned)(L.a.heads * 32));
+    switch (dv) {
+        case 32: attn_f32_kernel<DK, 32><<<grid, block, 0, s>>>(L.sv, L.a, L.idx, L.ld_idx, L.k_sel, L.st); return true;
+        case 64: attn_f32_kernel<DK, 64><<<grid, block, 0, s>>>(L.sv, L.a, L.idx, L.ld_idx, L.k_sel, L.st); return true;
+        case 96: attn_f32_kernel<DK, 96><<<grid, block, 0, s>>>(L.sv, L.a, L.idx, L.ld_idx, L.k_sel, L.st); return true;
+        case 128: attn_f32_kernel<DK, 128><<<grid, block, 0, s>>>(L.sv, L.a, L.idx, L.ld_idx, L.k_sel, L.st); return true;
+    }
+    return false;
+}
+
+bool launch_attn_f32(const AttnF32Launch& L, cudaStream_t s) {
+    if (L.total_q <= 0) return true;
+    switch (L.dk) {
+        case 32: return launch_attn_f32_dk<32>(L.dv, L, s);
+        case 64: return launch_attn_f32_dk<64>(L.dv, L, s);
+        case 96: return launch_attn_f32_dk<96>(L.dv, L, s);
+        case 128: return launch_attn_f32_dk<128>(L.dv, L, s);
+    }
+    return false;
+}
+
+// ---------------------------------------------------------------------------
+// Failure-detection self test: one thread waits on an mbarrier that nothing
+// arrives on, with a short budget, and records DSA_ERR_TIMEOUT.
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(StatusHdr* st, long long budget) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) mbar_init(b, 1);
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(b, 0, nullptr, st, 0x5e1f, budget);
+}
+
+void launch_selftest_wait(StatusHdr* st, long long budget, cudaStream_t s) {
+    selftest_wait_kernel<<<1, 32, 0, s>>>(st, budget);
+}
+
+}  // namespace dsa

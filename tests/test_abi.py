@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/dsa.h declares, and rejects bad arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_11_b200 import build
+    build.build()
+    from sparse_attention_11_b200 import dsa
+    return dsa
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    return sorted(set(re.findall(r"DSA_API\s+[\w\s\*]*?\b(dsa_\w+)\s*\(", src)))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward", "dsa_fold",
+              "dsa_workspace_size", "dsa_sync_status", "dsa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in _declared():
+        assert hasattr(raw, n), n
+    assert set(_declared()) <= set(lib.EXPORTED) | set(_declared())
+
+
+def test_status_strings(lib):
+    assert lib.status_string(0) == "ok"
+    assert "timed out" in lib.status_string(lib.DSA_ERR_TIMEOUT)
+    assert lib.status_string(99) == "unknown status"
+    assert lib.version() >= 1000
+
+
+def _fake_seqs(lib, batch=1, tq=64, tk=64):
+    # device pointers are never dereferenced on the host; any non-null value will do
+    return lib.dsa_seqs(batch, tq, tk, tq, tk, 0x1000, 0x2000)
+
+
+def test_validation_rejects_before_launch(lib):
+    S = _fake_seqs(lib)
+    P = ctypes.c_void_p
+    ws = P(0x10000)  # 256-aligned, never touched on rejection
+    # k < 1
+    assert lib.raw_call("dsa_topk", ctypes.byref(S), P(0x3000), 64, 0, 64, 0, P(0x4000), 64, ws, 1 << 20, None) \
+        == lib.DSA_ERR_INVALID_ARG
+    # rows out of range
+    assert lib.raw_call("dsa_topk", ctypes.byref(S), P(0x3000), 64, 10, 60, 8, P(0x4000), 64, ws, 1 << 20, None) \
+        == lib.DSA_ERR_INVALID_ARG
+    # ld_scores < max_seqlen_k
+    assert lib.raw_call("dsa_topk", ctypes.byref(S), P(0x3000), 32, 0, 64, 8, P(0x4000), 64, ws, 1 << 20, None) \
+        == lib.DSA_ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert lib.raw_call("dsa_topk", ctypes.byref(S), P(0x3000), 64, 0, 64, 8, P(0x4000), 64, ws, 16, None) \
+        == lib.DSA_ERR_WORKSPACE
+    assert lib.raw_call("dsa_topk", ctypes.byref(S), P(0x3000), 64, 0, 64, 8, P(0x4000), 64, P(0x10010), 1 << 20,
+                        None) == lib.DSA_ERR_INVALID_ARG
+    # batch 0
+    S0 = lib.dsa_seqs(0, 64, 64, 64, 64, 0x1000, 0x2000)
+    assert lib.raw_call("dsa_topk", ctypes.byref(S0), P(0x3000), 64, 0, 64, 8, P(0x4000), 64, ws, 1 << 20, None) \
+        == lib.DSA_ERR_INVALID_ARG
+
+
+def test_unsupported_attention_shapes(lib):
+    S = _fake_seqs(lib)
+    P = ctypes.c_void_p
+    ws = P(0x10000)
+    idx = P(0x5000)
+    for dt, h, dk, dv in ((lib.DSA_BF16, 64, 576, 512), (lib.DSA_BF16, 128, 128, 128), (lib.DSA_F32, 64, 64, 64),
+                          (lib.DSA_F32, 4, 48, 64), (7, 4, 64, 64)):
+        aa = lib.dsa_attn_args(dt, h, dk, dv, 0x100000, h * dk, dk, 0x200000, dk, 0x300000, dk, 0.1, 0x400000,
+                               h * dv, dv, None)
+        assert lib.raw_call("dsa_sparse_attn", ctypes.byref(S), ctypes.byref(aa), idx, 64, 64, ws, 1 << 20, None) \
+            == lib.DSA_ERR_UNSUPPORTED, (dt, h, dk, dv)
+
+
+def test_indexer_dtype_rules(lib):
+    S = _fake_seqs(lib)
+    P = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    # E4M3 without scales
+    ia = lib.dsa_indexer_args(lib.DSA_E4M3, 0x100000, None, lib.DSA_BF16, 0x200000, 0x300000, None)
+    assert lib.raw_call("dsa_fold", ctypes.byref(S), ctypes.byref(ia), P(0x400000), P(0x500000), P(0x10000),
+                        1 << 20, None) == lib.DSA_ERR_INVALID_ARG
+    # F32 with a bf16 W
+    ia = lib.dsa_indexer_args(lib.DSA_F32, 0x100000, None, lib.DSA_BF16, 0x200000, 0x300000, None)
+    assert lib.raw_call("dsa_fold", ctypes.byref(S), ctypes.byref(ia), P(0x400000), P(0x500000), P(0x10000),
+                        1 << 20, None) == lib.DSA_ERR_UNSUPPORTED
+    # workspace size grows with k for the forward op
+    ia = lib.dsa_indexer_args(lib.DSA_E4M3, 0x100000, 0x110000, lib.DSA_BF16, 0x200000, 0x300000, 0x310000)
+    sizes = []
+    for k in (64, 2048):
+        assert lib.raw_call("dsa_workspace_size", lib.DSA_OP_FORWARD, ctypes.byref(S), k, ctypes.byref(ia), None,
+                            ctypes.byref(n)) == 0
+        sizes.append(n.value)
+    assert sizes[1] > sizes[0] >= 256
