@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload prefill_l32768]
+
+One step = one pass of the whole path over one batch: fold W_index into the
+indexer queries, fused FP8 indexer + exact top-2048 (scores stay on chip),
+sparse MQA attention over the selected rows.  The headline workload is the
+L=32768 prefill (tokens/s); the same line carries the decode measurement
+(batch 64, contexts 16K-64K; tokens/s = 64 / step time).  Inputs are
+synthetic and seeded (sparse_attention_11_b200.workloads) and larger than
+L2, so no flush is needed between steps.
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload (the path shards by independent sequences; no collective on the
+data path); value = all ranks' tokens / max-over-ranks device time.
+
+--impl reference times the CPU oracle (oracle/), as it stands, on the host
+cores on a bounded stratified sample of the same workload.
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA prefill tokens/s at L=32K (indexer+top-2048+sparse attn); decode tok/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="prefill_l32768")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index):
+        import torch
+        self.ident = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            u = str(getattr(props, "uuid", ""))
+            if u:
+                self.ident = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            self.ident = None
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.ident:
+            cmd += ["-i", self.ident]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < len(self.FIELDS):
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                    pw.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # samples under load: power above half of the run's maximum
+        pmax = max(pw) if pw else 0
+        loaded = [s for s, p in zip(sm, pw) if p >= 0.5 * pmax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": pmax}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws, device=None):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workloads
+def workload_info(wl):
+    import numpy as np
+    pos = []
+    for sq, sk in zip(wl.seqlens_q, wl.seqlens_k):
+        pos.append(np.arange(sk - sq, sk, dtype=np.int64))
+    pos = np.concatenate(pos)
+    sel = np.minimum(pos + 1, wl.k)
+    return {"tokens": int(wl.total_q), "sum_sel": int(sel.sum()), "pairs": int((pos + 1).sum())}
+
+
+def attn_flops(wl, info):
+    return 2.0 * wl.heads * (wl.dk + wl.dv) * info["sum_sel"]
+
+
+def attn_bytes(wl, info):
+    """Algorithmic HBM bytes of one attention launch: gathered KV rows (V is the
+    latent part of K, so a row is dk bf16), q, out, lse, idx."""
+    row = wl.dk * 2 if wl.v_in_k else (wl.dk + wl.dv) * 2
+    return info["sum_sel"] * row + wl.total_q * wl.heads * (wl.dk + wl.dv) * 2 + wl.total_q * wl.heads * 4 + \
+        wl.total_q * wl.k * 4
+
+
+def run_native_workload(wl, steps, warmup, ws_n, rank, sampler=None):
+    """Device-timed steps of select + attention on one workload."""
+    import torch
+    from sparse_attention_11_b200 import dsa, workloads as W
+    from sparse_attention_11_b200.problem import DeviceProblem
+    inp = W.generate(wl, device="cuda")
+    prob = DeviceProblem(inp)
+    st = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(st)
+        dsa.dsa_select(prob.seqs, prob.ia, wl.k, prob.idx, prob.ws)
+        if evs:
+            evs[1].record(st)
+        dsa.dsa_sparse_attn(prob.seqs, prob.aa, prob.idx, wl.k, prob.ws)
+        if evs:
+            evs[2].record(st)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    prob.check("warmup")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    t0.record(st)
+    for i in range(steps):
+        step(evs[i])
+    t1.record(st)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier(ws_n)
+    prob.check("timed steps")
+    ms = t0.elapsed_time(t1)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    return inp, prob, ms, sel_ms, att_ms, clocks
+
+
+def e2e_native(inp, prob, steps):
+    """The same metric through dsa_forward with host inputs: every step copies
+    its inputs from pinned host memory and reads the attention output back."""
+    import torch
+    from sparse_attention_11_b200 import dsa
+    dev_tensors = [prob.q, prob.K, prob.q_idx, prob.k_idx, prob.W] + \
+        [t for t in (prob.q_idx_scale, prob.k_idx_scale) if t is not None]
+    if prob.V.data_ptr() != prob.K.data_ptr():
+        dev_tensors.append(prob.V)
+    host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in dev_tensors]
+    for h, d in zip(host, dev_tensors):
+        h.copy_(d)
+    out_host = torch.empty(prob.out.shape, dtype=prob.out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = out_host.numel() * out_host.element_size()
+    st = torch.cuda.current_stream()
+
+    def step():
+        for h, d in zip(host, dev_tensors):
+            d.copy_(h, non_blocking=True)
+        dsa.dsa_forward(prob.seqs, prob.ia, prob.aa, prob.wl.k, prob.idx, prob.ws)
+        out_host.copy_(prob.out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for _ in range(steps):
+        step()
+    t1.record(st)
+    torch.cuda.synchronize()
+    prob.check("e2e")
+    return t0.elapsed_time(t1) / steps, h2d, d2h
+
+
+def cpu_baseline(inp, target_s, max_rows=4096):
+    """The oracle, as it stands, on a stratified sample of query rows."""
+    import oracle
+    wl = inp.wl
+    T = wl.total_q
+    thr = oracle.num_threads()
+
+    def rows_for(n):
+        n = max(1, min(n, T))
+        return np.unique(np.linspace(0, T - 1, n).round().astype(np.int64))
+
+    def run(rows):
+        kb, pos = inp.key_base_pos(rows)
+        q = inp.q_rows(rows)
+        qs = inp.q_idx_scale[rows] if inp.q_idx_scale is not None else None
+        V = inp.K if inp.V is None else inp.V
+        vs = wl.dk if inp.V is None else wl.dv
+        t = time.perf_counter()
+        oracle.forward_rows(inp.q_idx[rows], qs, inp.W, inp.k_idx, inp.k_idx_scale, kb, pos, wl.k, q,
+                            inp.K.ravel(), wl.dk, V.ravel(), vs, wl.scale, wl.dv)
+        return time.perf_counter() - t
+
+    cal = rows_for(thr)
+    t_cal = run(cal)
+    n = int(min(max_rows, max(len(cal), len(cal) * target_s / max(t_cal, 1e-3))))
+    rows = rows_for(n)
+    t = run(rows)
+    return {"value": len(rows) / t, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{len(rows)} query rows of {wl.name} evenly spaced over all positions "
+                      f"(fold, scores, top-{wl.k}, attention per row), {t:.1f} s; tokens/s = rows/s",
+            "seconds": t}
+
+
+# ----------------------------------------------------------------------------- native arm
+def native(args):
+    import torch
+    from sparse_attention_11_b200 import workloads as W
+    ws_n, rank, local = dist_setup(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    wl = W.WORKLOADS[args.workload]
+    info = workload_info(wl)
+    sampler = ClockSampler(torch.cuda.current_device())
+    inp, prob, ms, sel_ms, att_ms, clocks = run_native_workload(wl, args.steps, args.warmup, ws_n, rank, sampler)
+    ms_max = max_over_ranks(ms, ws_n, dev)
+    tokens_per_step = info["tokens"]
+    value = ws_n * tokens_per_step * args.steps / (ms_max / 1e3)
+    att_max = max_over_ranks(att_ms, ws_n, dev)
+    flops = attn_flops(wl, info)
+    achieved_tf = flops / (att_max / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "dtypes": {"indexer": "e4m3", "attention": "bf16", "accumulate": "f32"},
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "seq_len": int(max(wl.seqlens_k)), "top_k": wl.k,
+                   "heads": wl.heads, "dk": wl.dk, "dv": wl.dv, "v": "latent part of K" if wl.v_in_k else "own tensor",
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws_n}"},
+        "stages_ms": {"select": sel_ms, "attention": att_ms},
+        "roofline": {"kernel": "attn_tc_kernel", "bound": "tensor", "achieved": achieved_tf,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved_tf / peak,
+                     "peak_kind": f"bf16 {peaks['source']} sustained", "flops_per_launch": flops,
+                     "frac_of_burst": achieved_tf / peaks["bf16_tflops"], "traffic": None},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    traffic = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(traffic):
+        with open(traffic) as f:
+            tr = json.load(f).get(wl.name, {}).get("attn_tc_kernel")
+        if tr:
+            res["roofline"]["traffic"] = tr["bytes_per_launch"]
+            res["roofline"]["traffic_source"] = tr["source"]
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_native(inp, prob, max(1, min(args.steps, 5)))
+        e2e_max = max_over_ranks(e2e_ms, ws_n, dev)
+        res["e2e"] = {"value": ws_n * tokens_per_step / (e2e_max / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max, "api": "dsa_forward"}
+    if not args.no_decode and wl.name != "decode_b64":
+        del prob
+        torch.cuda.empty_cache()
+        dwl = W.WORKLOADS["decode_b64"]
+        dinfo = workload_info(dwl)
+        dsteps = max(args.steps, 20)
+        dinp, dprob, dms, dsel, datt, _ = run_native_workload(dwl, dsteps, args.warmup, ws_n, rank, None)
+        dms_max = max_over_ranks(dms, ws_n, dev)
+        datt_max = max_over_ranks(datt, ws_n, dev)
+        byts = attn_bytes(dwl, dinfo)
+        scan_bytes = dinfo["pairs"] * 132
+        res["decode"] = {
+            "workload": dwl.name, "value": ws_n * dinfo["tokens"] * dsteps / (dms_max / 1e3), "unit": "tokens/s",
+            "ms_per_step": dms_max / dsteps, "steps": dsteps, "stages_ms": {"select": dsel, "attention": datt},
+            "roofline": {"kernel": "attn_tc_kernel", "bound": "hbm", "achieved": byts / (datt_max / 1e3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": byts / (datt_max / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_launch": byts},
+            "select_hbm": {"bytes_scan": scan_bytes, "achieved_gbs": scan_bytes / (dsel / 1e3) / 1e9},
+            "gpu_launches": 5 * dsteps,
+        }
+        if not args.no_e2e:
+            e2e_ms, h2d, d2h = e2e_native(dinp, dprob, 5)
+            res["decode"]["e2e"] = {"value": ws_n * dinfo["tokens"] / (max_over_ranks(e2e_ms, ws_n, dev) / 1e3),
+                                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del dprob
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+def reference(args):
+    ws_n = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from sparse_attention_11_b200 import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    inp = W.generate(wl, device="cpu", q_on_device=False) if wl.attn_dtype == "f32" else None
+    if inp is None:
+        # the attention queries are drawn on the GPU; without one, draw them on the CPU generator
+        import torch
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        inp = W.generate(wl, device=dev)
+    per_step_s = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(inp, per_step_s / 4)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = cpu_baseline(inp, per_step_s)
+        vals.append(r["value"])
+        secs.append(r["seconds"])
+    v = statistics.median(vals)
+    res = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": wl.name, "batch": wl.batch, "seq_len": int(max(wl.seqlens_k)), "top_k": wl.k,
+                      "heads": wl.heads, "dk": wl.dk, "dv": wl.dv},
+           "cpu_baseline": {"kind": "oracle", "cores": r["cores"], "sample": r["sample"], "value": v},
+           "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference(args)
+    else:
+        native(args)
+
+
+if __name__ == "__main__":
+    main()

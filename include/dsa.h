@@ -176,6 +176,14 @@ DSA_API int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_score
 DSA_API int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx,
                     int64_t ld_idx, int32_t k_sel, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* Steps a1-a3 -- fold, then the fused indexer/top-k: idx (int32
+ * [total_q, ld_idx], ld_idx >= k) receives, for every query, its
+ * K_t = min(k, pos+1) selected keys in ascending index order followed by -1
+ * (the selection dsa_topk makes on the scores of dsa_index_scores).  The
+ * L x L scores are never written to memory.  Workspace: DSA_OP_FORWARD. */
+DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
+                       int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
 /* The whole hot path: a1 fold -> a2+a3 fused indexer/top-k (the scores stay
  * on chip) -> a4 sparse attention.  idx_out (nullable; int32
  * [total_q, ld_idx]) receives the selected indices as dsa_topk would

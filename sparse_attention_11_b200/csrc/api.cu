@@ -371,6 +371,36 @@ int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t
     return run_attn(seqs, aa, idx, ld_idx, k_sel, hdr(ws), (cudaStream_t)stream);
 }
 
+namespace {
+int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx, int64_t ldi,
+                const WsLayout& L, void* ws, cudaStream_t st) {
+    uint8_t* w = (uint8_t*)ws;
+    int r = run_fold(seqs, ia, w + L.u, (float*)(w + L.s_row), st);
+    if (r) return r;
+    if (use_tc_indexer(seqs, ia))
+        return run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, k, idx, ldi, nullptr, 0, 0, 0, hdr(ws),
+                              st);
+    float* sc = (float*)(w + L.scores);
+    const int64_t ld = seqs->max_seqlen_k;
+    r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st);
+    if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st);
+    return r;
+}
+}  // namespace
+
+int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx, int64_t ld_idx, void* ws,
+               size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_indexer(seqs, ia);
+    if (r) return r;
+    if (k < 1 || (seqs->total_q && (!idx || ld_idx < k))) return DSA_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia));
+    r = check_ws(ws, ws_bytes, L.total);
+    if (r) return r;
+    if (seqs->total_q == 0) return DSA_OK;
+    return select_into(seqs, ia, k, idx, ld_idx, L, ws, (cudaStream_t)stream);
+}
+
 int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k, int32_t* idx_out,
                 int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
     int r = check_seqs(seqs);
@@ -379,25 +409,14 @@ int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn
     if (r) return r;
     if (k < 1) return DSA_ERR_INVALID_ARG;
     if (idx_out && ld_idx < k) return DSA_ERR_INVALID_ARG;
-    const bool tc = use_tc_indexer(seqs, ia);
-    const WsLayout L = ws_layout(seqs, ia, k, true, !tc);
+    const WsLayout L = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia));
     r = check_ws(ws, ws_bytes, L.total);
     if (r) return r;
     if (seqs->total_q == 0) return DSA_OK;
     cudaStream_t st = (cudaStream_t)stream;
-    uint8_t* w = (uint8_t*)ws;
-    int32_t* idx = idx_out ? idx_out : (int32_t*)(w + L.idx);
+    int32_t* idx = idx_out ? idx_out : (int32_t*)((uint8_t*)ws + L.idx);
     const int64_t ldi = idx_out ? ld_idx : k;
-    r = run_fold(seqs, ia, w + L.u, (float*)(w + L.s_row), st);
-    if (r) return r;
-    if (tc) {
-        r = run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, k, idx, ldi, nullptr, 0, 0, 0, hdr(ws), st);
-    } else {
-        float* sc = (float*)(w + L.scores);
-        const int64_t ld = seqs->max_seqlen_k;
-        r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st);
-        if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st);
-    }
+    r = select_into(seqs, ia, k, idx, ldi, L, ws, st);
     if (r) return r;
     return run_attn(seqs, aa, idx, ldi, k, hdr(ws), st);
 }

@@ -13,11 +13,17 @@
 //   rank 1: contraction columns [256,576) output columns [256,512)
 // When V is the latent part of K (V = K[:, :512]) each CTA's V columns are
 // the first 256 of its own K columns, so every gathered byte is used once.
-// Per 64-key tile each CTA computes a partial S; the pair exchanges halves
-// over DSMEM (rank 0 finishes the softmax of heads 0..63, rank 1 of
-// 64..127), then exchanges the bf16 probabilities, and each CTA accumulates
-// its half of O.  Online softmax with lazy rescaling (the running max is
-// only moved when it grows by more than 2^8).
+//
+// Softmax split: per 64-key tile each CTA holds a partial S for all 128 heads
+// and all 64 keys.  Rank r finishes the scores of keys [32r, 32r+32) for all
+// heads: it sends the other 32 partial columns to its peer and receives the
+// peer's partials of its own 32 keys (st.async into the peer's shared memory,
+// counted on the peer's mbarrier).  Both CTAs use the same running maximum:
+// the sum of the two partial maxima of the tile, an upper bound of the true
+// maximum that both can form from the exchanged data, with lazy rescaling
+// (moved only when it grows by more than 2^8).  Each CTA then computes bf16
+// probabilities for its 32 keys, sends them to the peer, and accumulates its
+// half of O over all 64 keys.  The row sums are combined once at the end.
 //
 // Tensor memory per CTA (512 columns): O [0,256)  S [256,320)  P [320,352)
 // Q [352, 352 + 32 * blocks).  Q and P are the A operands, read from TMEM
@@ -35,16 +41,19 @@ constexpr int AT_N = 64;                            // keys per tile
 constexpr uint32_t AT_BLK = AT_N * 128;             // one 64-column block of a tile
 constexpr uint32_t AT_KST = 5 * AT_BLK;             // K part of a stage (max 5 blocks)
 constexpr uint32_t AT_VST = 4 * AT_BLK;             // V part (separate V only)
-constexpr uint32_t AT_SX_PITCH = 272;               // 64 fp32 + pad
-constexpr uint32_t AT_PX_PITCH = 144;               // 64 bf16 + (alpha, l) + pad
+constexpr uint32_t AT_SX_PITCH = 144;               // 32 fp32 partials + partial max + pad
+constexpr uint32_t AT_PX_PITCH = 80;                // 32 bf16 probabilities + pad
+constexpr uint32_t AT_SX_BYTES = 128 * 9 * 16;      // bytes counted per tile
+constexpr uint32_t AT_PX_BYTES = 128 * 4 * 16;
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_P = 320, TM_Q = 352;
 
 template <int NST, bool VSEP>
 struct AtLayout {
     static constexpr uint32_t STAGE = AT_KST + (VSEP ? AT_VST : 0);
-    static constexpr uint32_t OFF_SX = NST * STAGE;
-    static constexpr uint32_t OFF_PX = OFF_SX + 64 * AT_SX_PITCH;
-    static constexpr uint32_t OFF_BAR = OFF_PX + 64 * AT_PX_PITCH;
+    static constexpr uint32_t OFF_SX = NST * STAGE;                   // [2][128][144]
+    static constexpr uint32_t OFF_PX = OFF_SX + 2 * 128 * AT_SX_PITCH;  // [2][128][80]
+    static constexpr uint32_t OFF_LX = OFF_PX + 2 * 128 * AT_PX_PITCH;  // [128] fp32
+    static constexpr uint32_t OFF_BAR = OFF_LX + 512;
     static constexpr uint32_t SMEM = OFF_BAR + 512 + 1024;
 };
 
@@ -52,7 +61,8 @@ struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
     uint64_t s_full, s_empty, p_full, p_free, q_full, o_full;
-    uint64_t sx_full, sx_free, px_full, px_free;  // arrived on by the peer CTA
+    uint64_t sx_full[2], px_full[2], lx_full;  // filled by the peer (st.async, byte-counted)
+    uint64_t sx_free[2], px_free[2];           // the peer consumed what this CTA sent
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -92,11 +102,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         mbar_init(smem_u32(&bars->p_free), 1);
         mbar_init(smem_u32(&bars->q_full), 4);
         mbar_init(smem_u32(&bars->o_full), 1);
-        mbar_init(smem_u32(&bars->sx_full), 2);
-        mbar_init(smem_u32(&bars->sx_free), 2);
-        mbar_init(smem_u32(&bars->px_full), 2);
-        mbar_init(smem_u32(&bars->px_free), 2);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bars->sx_full[i]), 1);
+            mbar_init(smem_u32(&bars->px_full[i]), 1);
+            mbar_init(smem_u32(&bars->sx_free[i]), 4);
+            mbar_init(smem_u32(&bars->px_free[i]), 4);
+        }
+        mbar_init(smem_u32(&bars->lx_full), 1);
         mbar_init(smem_u32(&bars->drain), 1);
+        // arm the byte-counted barriers for their first phase
+        for (int i = 0; i < 2; ++i) {
+            mbar_arrive_expect_tx(smem_u32(&bars->sx_full[i]), AT_SX_BYTES);
+            mbar_arrive_expect_tx(smem_u32(&bars->px_full[i]), AT_PX_BYTES);
+        }
+        mbar_arrive_expect_tx(smem_u32(&bars->lx_full), 128 * 4);
         bars->abort = 0;
         bars->max_slot = -1;
         fence_mbar_init();
@@ -112,7 +131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         if (lane == 0 && m >= 0) atomicMax(&bars->max_slot, m);
     }
     tc_fence_before();
-    cluster_sync();  // barriers of both CTAs initialised; max_slot final
+    cluster_sync();  // barriers of both CTAs initialised and armed; max_slot final
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const int n_tiles = (bars->max_slot + AT_N) / AT_N;
@@ -126,19 +145,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         }
         uint32_t last_issued[NST];
         for (int i = 0; i < NST; ++i) last_issued[i] = 0xFFFFFFFFu;
-        for (int j = 0; j < n_tiles; ++j) {
-            const uint32_t s = j % NST;
-            if (!wait_warp(smem_u32(&bars->empty[s]), ((j / NST) & 1) ^ 1, abort, st, 0x2101)) break;
-            int32_t rows[4];
+        int32_t nxt[4];
+        auto load_rows = [&](int j, int32_t (&rw)[4]) {
             if (lane < 16) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int slot = j * AT_N + lane * 4 + i;
-                    const int32_t v = slot < a.k_sel ? __ldg(irow + slot) : -1;
+                    rw[i] = slot < a.k_sel ? __ldg(irow + slot) : -1;
+                }
+            }
+        };
+        if (n_tiles > 0) load_rows(0, nxt);
+        for (int j = 0; j < n_tiles; ++j) {
+            const uint32_t s = j % NST;
+            int32_t rows[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rows[i] = nxt[i];
+            if (j + 1 < n_tiles) load_rows(j + 1, nxt);
+            if (lane < 16) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int32_t v = rows[i];
                     if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
                     rows[i] = (int32_t)(ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0));
                 }
             }
+            if (!wait_warp(smem_u32(&bars->empty[s]), ((j / NST) & 1) ^ 1, abort, st, 0x2101)) break;
             if (lane == 0)
                 mbar_arrive_expect_tx(smem_u32(&bars->full[s]), nb * AT_BLK + (VSEP ? AT_VST : 0));
             __syncwarp();
@@ -207,17 +239,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         // ================= softmax / exchange / epilogue =================
         const uint32_t quad = warp & 3;
         const int h = (int)(quad * 32 + lane);
-        const bool owner = (quad >> 1) == rank;
         const uint32_t lane_off = (quad * 32) << 16;
-        const int xrow = h & 63;
+        const int kh = (int)rank;             // this CTA's key half of every tile
         uint8_t* sx = smem + Lay::OFF_SX;
         uint8_t* px = smem + Lay::OFF_PX;
+        float* lx = (float*)(smem + Lay::OFF_LX);
         const uint32_t peer_sx = mapa(smem_u32(sx), peer);
         const uint32_t peer_px = mapa(smem_u32(px), peer);
-        const uint32_t peer_sx_full = mapa(smem_u32(&bars->sx_full), peer);
-        const uint32_t peer_sx_free = mapa(smem_u32(&bars->sx_free), peer);
-        const uint32_t peer_px_full = mapa(smem_u32(&bars->px_full), peer);
-        const uint32_t peer_px_free = mapa(smem_u32(&bars->px_free), peer);
+        const uint32_t peer_lx = mapa(smem_u32(lx), peer);
+        // peer barrier addresses of buffer b are base + 8 b (same layout in both CTAs)
+        const uint32_t peer_sx_full0 = mapa(smem_u32(&bars->sx_full[0]), peer);
+        const uint32_t peer_px_full0 = mapa(smem_u32(&bars->px_full[0]), peer);
+        const uint32_t peer_sx_free0 = mapa(smem_u32(&bars->sx_free[0]), peer);
+        const uint32_t peer_px_free0 = mapa(smem_u32(&bars->px_free[0]), peer);
+        const uint32_t my_sx_full0 = smem_u32(&bars->sx_full[0]), my_px_full0 = smem_u32(&bars->px_full[0]);
+        const uint32_t my_sx_free0 = smem_u32(&bars->sx_free[0]), my_px_free0 = smem_u32(&bars->px_free[0]);
+        const uint32_t peer_lx_full = mapa(smem_u32(&bars->lx_full), peer);
+        const bool arm_thread = threadIdx.x == 64;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
@@ -238,96 +276,108 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
         }
+        int32_t nv0 = -1, nv1 = -1;
+        if (n_tiles > 0) {
+            nv0 = lane < a.k_sel ? __ldg(irow + lane) : -1;
+            nv1 = lane + 32 < a.k_sel ? __ldg(irow + lane + 32) : -1;
+        }
         for (int j = 0; ok && j < n_tiles; ++j) {
-            // validity of this tile's 64 slots
-            const int sl0 = j * AT_N + lane, sl1 = sl0 + 32;
-            const int32_t v0 = sl0 < a.k_sel ? __ldg(irow + sl0) : -1;
-            const int32_t v1 = sl1 < a.k_sel ? __ldg(irow + sl1) : -1;
+            const uint32_t b = j & 1, ph = (j >> 1) & 1;
+            const int32_t v0 = nv0, v1 = nv1;
+            if (j + 1 < n_tiles) {  // prefetch the next tile's slots
+                const int sl0 = (j + 1) * AT_N + lane, sl1 = sl0 + 32;
+                nv0 = sl0 < a.k_sel ? __ldg(irow + sl0) : -1;
+                nv1 = sl1 < a.k_sel ? __ldg(irow + sl1) : -1;
+            }
             const uint32_t mlo = __ballot_sync(0xffffffffu, v0 >= 0 && v0 < ri.seqlen_k);
             const uint32_t mhi = __ballot_sync(0xffffffffu, v1 >= 0 && v1 < ri.seqlen_k);
+            const uint32_t mine = kh ? mhi : mlo;      // validity of this CTA's 32 keys
             if (!wait_warp(smem_u32(&bars->s_full), j & 1, abort, st, 0x2301)) { ok = false; break; }
             tc_fence_after();
-            float sv[64];
+            float sa[64];
             {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + TM_S, r);
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + TM_S, r0);
+                tmem_ld32(tmem + lane_off + TM_S + 32, r1);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r[i]);
-                tmem_ld32(tmem + lane_off + TM_S + 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) {
+                    sa[i] = __uint_as_float(r0[i]);
+                    sa[32 + i] = __uint_as_float(r1[i]);
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
-            uint32_t praw[32];
-            float alpha = 1.f;
-            if (!owner) {
-                // send my partial S of the peer's heads
-                if (!wait_warp(smem_u32(&bars->sx_free), (j & 1) ^ 1, abort, st, 0x2302)) { ok = false; break; }
-                const uint32_t dst = peer_sx + xrow * AT_SX_PITCH;
+            // partial maximum over the tile's valid keys
+            float pm = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    st_cluster_v4(dst + c * 16, __float_as_uint(sv[4 * c]), __float_as_uint(sv[4 * c + 1]),
-                                  __float_as_uint(sv[4 * c + 2]), __float_as_uint(sv[4 * c + 3]));
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(peer_sx_full);
-                // receive the peer's probabilities for these heads
-                if (!wait_warp_cluster(smem_u32(&bars->px_full), j & 1, abort, st, 0x2303)) { ok = false; break; }
-                const uint4* src = (const uint4*)(px + xrow * AT_PX_PITCH);
+            for (int i = 0; i < 32; ++i) {
+                if ((mlo >> i) & 1u) pm = fmaxf(pm, sa[i]);
+                if ((mhi >> i) & 1u) pm = fmaxf(pm, sa[32 + i]);
+            }
+            // send the peer's 32 partial columns and the partial max
+            if (!wait_warp_cluster(my_sx_free0 + 8 * b, ph ^ 1, abort, st, 0x2302)) { ok = false; break; }
+            {
+                const uint32_t dst = peer_sx + b * (128 * AT_SX_PITCH) + h * AT_SX_PITCH;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 v = src[c];
-                    praw[4 * c] = v.x; praw[4 * c + 1] = v.y; praw[4 * c + 2] = v.z; praw[4 * c + 3] = v.w;
-                }
-                const uint4 tail = src[8];
-                alpha = __uint_as_float(tail.x);
-                l = __uint_as_float(tail.y);
-            } else {
-                // combine with the peer's partial S of my heads
-                if (!wait_warp_cluster(smem_u32(&bars->sx_full), j & 1, abort, st, 0x2304)) { ok = false; break; }
-                const float4* src = (const float4*)(sx + xrow * AT_SX_PITCH);
+                    // the peer's keys: [32, 64) for rank 0, [0, 32) for rank 1
+                    uint32_t w[4];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
+                    for (int e = 0; e < 4; ++e) w[e] = __float_as_uint(kh ? sa[4 * c + e] : sa[32 + 4 * c + e]);
+                    st_async_v4(dst + c * 16, w[0], w[1], w[2], w[3], peer_sx_full0 + 8 * b);
+                }
+                st_async_v4(dst + 128, __float_as_uint(pm), 0u, 0u, 0u, peer_sx_full0 + 8 * b);
+            }
+            // receive the peer's partials of this CTA's 32 keys
+            if (!wait_warp_cluster(my_sx_full0 + 8 * b, ph, abort, st, 0x2303)) { ok = false; break; }
+            if (arm_thread && j + 2 < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * b, AT_SX_BYTES);
+            float s32[32];
+            float pm_peer;
+            {
+                const float4* src = (const float4*)(sx + b * (128 * AT_SX_PITCH) + h * AT_SX_PITCH);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
                     const float4 v = src[c];
-                    sv[4 * c] += v.x; sv[4 * c + 1] += v.y; sv[4 * c + 2] += v.z; sv[4 * c + 3] += v.w;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(peer_sx_free);
-                // online softmax (base 2), lazy rescaling
-                float mx = -INFINITY;
+                    const float pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const bool valid = ((i < 32 ? mlo >> i : mhi >> (i - 32)) & 1u) != 0;
-                    sv[i] = valid ? sv[i] * a.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, sv[i]);
+                    for (int e = 0; e < 4; ++e) s32[4 * c + e] = (kh ? sa[32 + 4 * c + e] : sa[4 * c + e]) + pv[e];
                 }
-                if (mx > m_used + 8.0f) {
-                    alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mx);
-                    l *= alpha;
-                    m_used = mx;
-                }
+                pm_peer = src[8].x;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * b);
+            // shared running maximum (identical in both CTAs), lazy rescale
+            const float mb = (pm == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm + pm_peer) * a.scale_log2;
+            float alpha = 1.f;
+            if (mb > m_used + 8.0f) {
+                alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mb);
+                l *= alpha;
+                m_used = mb;
+            }
+            uint32_t pw[16];
+            {
                 float rs = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float p0 = m_used == -INFINITY ? 0.f : ex2(sv[2 * i] - m_used);
-                    const float p1 = m_used == -INFINITY ? 0.f : ex2(sv[2 * i + 1] - m_used);
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = ((mine >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
+                    const float p1 = ((mine >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
                     rs += p0 + p1;
-                    praw[i] = pack_bf16(p0, p1);
+                    pw[i] = pack_bf16(p0, p1);
                 }
                 l += rs;
-                if (!wait_warp_cluster(smem_u32(&bars->px_free), (j & 1) ^ 1, abort, st, 0x2305)) { ok = false; break; }
-                const uint32_t dst = peer_px + xrow * AT_PX_PITCH;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) st_cluster_v4(dst + c * 16, praw[4 * c], praw[4 * c + 1], praw[4 * c + 2], praw[4 * c + 3]);
-                st_cluster_v4(dst + 128, __float_as_uint(alpha), __float_as_uint(l), 0u, 0u);
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(peer_px_full);
             }
-            // O rescale and P -> TMEM once the previous P.V has finished
-            if (!wait_warp(smem_u32(&bars->p_free), (j & 1) ^ 1, abort, st, 0x2306)) { ok = false; break; }
+            // send this CTA's probabilities to the peer
+            if (!wait_warp_cluster(my_px_free0 + 8 * b, ph ^ 1, abort, st, 0x2304)) { ok = false; break; }
+            {
+                const uint32_t dst = peer_px + b * (128 * AT_PX_PITCH) + h * AT_PX_PITCH;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    st_async_v4(dst + c * 16, pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3], peer_px_full0 + 8 * b);
+            }
+            // O rescale and this CTA's P half -> TMEM once the previous P.V is done
+            if (!wait_warp(smem_u32(&bars->p_free), (j & 1) ^ 1, abort, st, 0x2305)) { ok = false; break; }
             tc_fence_after();
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 for (int c = 0; c < 8; ++c) {
@@ -339,20 +389,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
                     tmem_st32(tmem + lane_off + TM_O + c * 32, r);
                 }
             }
-            tmem_st32(tmem + lane_off + TM_P, praw);
+            tmem_st16(tmem + lane_off + TM_P + 16 * kh, pw);
+            // the peer's P half
+            if (!wait_warp_cluster(my_px_full0 + 8 * b, ph, abort, st, 0x2306)) { ok = false; break; }
+            if (arm_thread && j + 2 < n_tiles) mbar_arrive_expect_tx(my_px_full0 + 8 * b, AT_PX_BYTES);
+            {
+                uint32_t r[16];
+                const uint4* src = (const uint4*)(px + b * (128 * AT_PX_PITCH) + h * AT_PX_PITCH);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = src[c];
+                    r[4 * c] = v.x; r[4 * c + 1] = v.y; r[4 * c + 2] = v.z; r[4 * c + 3] = v.w;
+                }
+                tmem_st16(tmem + lane_off + TM_P + 16 * (1 - kh), r);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(smem_u32(&bars->p_full));
-                if (!owner) mbar_arrive_remote(peer_px_free);
+                mbar_arrive_remote(peer_px_free0 + 8 * b);
             }
+        }
+        // ---- row sums of both halves ----
+        float l_tot = 0.f;
+        if (ok && n_tiles > 0) {
+            st_async_b32(peer_lx + h * 4, __float_as_uint(l), peer_lx_full);
+            if (wait_warp_cluster(smem_u32(&bars->lx_full), 0, abort, st, 0x2307)) l_tot = l + lx[h];
+            else ok = false;
         }
         // ---- epilogue: O / l -> bf16 ----
         __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0;
-        const bool have_o = ok && n_tiles > 0 && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2307);
+        const bool have_o = ok && n_tiles > 0 && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2308);
         if (have_o) tc_fence_after();
-        const float inv = l > 0.f ? 1.0f / l : 0.f;
+        const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
         for (int c = 0; c < 8; ++c) {
             uint32_t r[32];
             if (have_o) {
@@ -374,8 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
                 dst[i] = w;
             }
         }
-        if (owner && a.lse)
-            a.lse[t * 128 + h] = (have_o && l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (rank == 0 && a.lse)
+            a.lse[t * 128 + h] = (have_o && l_tot > 0.f) ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
     }
     tc_fence_before();
     __syncwarp();

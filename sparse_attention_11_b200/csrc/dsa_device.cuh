@@ -120,12 +120,14 @@ DSA_DEV bool mbar_wait_impl(uint32_t bar, uint32_t parity, volatile int* abort, 
     for (uint32_t it = 1;; ++it) {
         if (test()) return true;
         if (abort && *abort) return false;
-        if ((it & 63) == 0) {
-            if (st && *(volatile int*)&st->code == DSA_ERR_TIMEOUT) {
+        if ((it & 15) == 0) {
+            const long long el = clock64() - t0;
+            // the global header is only read once a wait is already long
+            if (el > (1ll << 20) && st && *(volatile int*)&st->code == DSA_ERR_TIMEOUT) {
                 if (abort) *abort = 1;
                 return false;
             }
-            if (clock64() - t0 > budget) {
+            if (el > budget) {
                 report(st, DSA_ERR_TIMEOUT, where);
                 if (abort) *abort = 1;
                 return false;
@@ -170,6 +172,18 @@ DSA_DEV void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, ui
     asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
+// Store into another CTA's shared memory and count the bytes on its
+// mbarrier (complete_tx): the data is visible once that phase completes.
+DSA_DEV void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
+                 : "memory");
+}
+DSA_DEV void st_async_b32(uint32_t addr, uint32_t a, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(a),
+                 "r"(remote_bar)
+                 : "memory");
+}
 DSA_DEV void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -185,6 +199,13 @@ DSA_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"((uint64_t)m), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+// Contiguous bytes global -> this CTA's shared memory (both 16-byte aligned,
+// size a multiple of 16), counted on `bar`.
+DSA_DEV void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"((uint64_t)src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 // Four rows y0..y3 of columns [x, x+box) into dst (4 consecutive box rows).
 DSA_DEV void tma_gather4(uint32_t dst, const CUtensorMap* m, int32_t x, int32_t y0, int32_t y1, int32_t y2, int32_t y3,
@@ -280,6 +301,21 @@ DSA_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
         "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
         "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+DSA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+DSA_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 

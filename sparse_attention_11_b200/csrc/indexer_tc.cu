@@ -64,6 +64,112 @@ struct IxBars {
     int abort;
 };
 
+// Scores of 32 consecutive columns as non-negative fp32 bit patterns,
+// computed in place: ReLU((dot * s_k) * s_row), +inf/NaN clamped to +inf.
+// The 32 lanes of work are independent so the chain latencies overlap.
+__device__ __forceinline__ void chunk_keys(uint32_t (&v)[32], const float* scs, float srow) {
+    const float4* s4 = (const float4*)scs;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 sk = s4[q];
+        const float skv[4] = {sk.x, sk.y, sk.z, sk.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x = __fmul_rn(__fmul_rn(__uint_as_float(v[4 * q + e]), skv[e]), srow);
+            v[4 * q + e] = (uint32_t)min(max(__float_as_int(x), 0), 0x7F800000);
+        }
+    }
+}
+
+// Per-row radix state of the epilogue thread.
+struct RowSel {
+    int sh, P;          // current bucket: keys with ((bits - 1) >> sh) == P
+    uint32_t need;      // keys still to take from the bucket
+    uint32_t taken;     // bucket keys taken so far in the emission sweep
+    int cnt;            // indices written
+    bool take_all;      // pos + 1 <= k: the whole causal prefix
+};
+
+// One 32-column chunk, columns c with c <= lim are causal.
+template <int MODE>  // SW_HIST level 1 (1), deeper level (4), SW_EMIT (2), SW_SCORES (3)
+__device__ __forceinline__ void ep_chunk(uint32_t (&v)[32], const float* scs, float srow, int lim, int32_t sbase,
+                                         RowSel& rs, uint32_t* myhist, int dshift, uint32_t dmask, int32_t* out, int kcap,
+                                         float* srow_out) {
+    chunk_keys(v, scs, srow);
+#define KB(i) ((int)v[i])
+    const uint32_t limmask = lim >= 31 ? 0xFFFFFFFFu : ((1u << (lim + 1)) - 1u);
+    if (MODE == 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if ((limmask >> i) & 1u) atomicAdd(&myhist[((uint32_t)KB(i) + 0x7FFFFFu) >> 23 << 7], 1u);
+    } else if (MODE == 4) {
+        uint32_t mem = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mem |= (uint32_t)(((KB(i) - 1) >> rs.sh) == rs.P) << i;
+        mem &= limmask;
+        while (mem) {
+            const int i = __ffs(mem) - 1;
+            mem &= mem - 1;
+            int ki = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ki = (e == i) ? KB(e) : ki;
+            atomicAdd(&myhist[(((uint32_t)(ki - 1) >> dshift) & dmask) << 7], 1u);
+        }
+    } else if (MODE == 2) {
+        uint32_t above = 0, eq = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int hi = (KB(i) - 1) >> rs.sh;
+            above |= (uint32_t)(hi > rs.P) << i;
+            eq |= (uint32_t)(hi == rs.P) << i;
+        }
+        if (rs.take_all) above = 0xFFFFFFFFu, eq = 0;
+        above &= limmask;
+        eq &= limmask;
+        uint32_t any = above | eq;
+        while (any) {
+            const int i = __ffs(any) - 1;
+            any &= any - 1;
+            bool e = (above >> i) & 1u;
+            if (!e && rs.taken < rs.need) {
+                e = true;
+                ++rs.taken;
+            }
+            if (e) {
+                if (rs.cnt < kcap) out[rs.cnt] = sbase + i;
+                ++rs.cnt;
+            }
+        }
+    } else if (MODE == 3) {
+        if (srow_out) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if ((limmask >> i) & 1u) srow_out[sbase + i] = __int_as_float(KB(i));
+        }
+    }
+}
+#undef KB
+
+// All 256 columns of a tile for one row, one 32-column TMEM load at a time.
+template <int MODE>
+__device__ __forceinline__ void ep_tile(uint32_t taddr, bool ok, bool active, const float* scs, float srow, int64_t pos,
+                                        int64_t s_tile, RowSel& rs, uint32_t* myhist, int dshift, uint32_t dmask,
+                                        int32_t* out, int kcap, float* srow_out) {
+#pragma unroll 1
+    for (int ch = 0; ch < 8; ++ch) {
+        uint32_t v[32];
+        if (ok) {
+            tmem_ld32(taddr + ch * 32, v);
+            tmem_wait_ld();
+        }
+        if (!active) continue;
+        const int64_t sb = s_tile + ch * 32;
+        if (sb <= pos)
+            ep_chunk<MODE>(v, scs + ch * 32, srow, (int)min((int64_t)31, pos - sb), (int32_t)sb, rs, myhist, dshift, dmask,
+                           out, kcap, srow_out);
+    }
+}
+
 __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constant__ IndexerTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -143,14 +249,19 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
                     if (!wait_warp(smem_u32(&bars->empty[s]), ((g / IX_NST) & 1) ^ 1, abort, st, 0x1101)) break;
                     const int64_t kr0 = key_base + (int64_t)tile * IX_BN;
                     float* scs = sc_s + s * IX_BN;
-                    for (int i = lane; i < IX_BN; i += 32) {
-                        const int64_t kr = kr0 + i;
-                        scs[i] = (tile * IX_BN + i <= pos_last) ? __ldg(a.k_scale + kr) : 0.f;
+                    // full tiles with 16-byte aligned scales: one bulk copy; else plain loads
+                    const bool bulk = (tile + 1) * IX_BN <= pos_last + 1 && ((uintptr_t)(a.k_scale + kr0) & 15) == 0;
+                    if (!bulk) {
+                        for (int i = lane; i < IX_BN; i += 32) {
+                            const int64_t kr = kr0 + i;
+                            scs[i] = (tile * IX_BN + i <= pos_last) ? __ldg(a.k_scale + kr) : 0.f;
+                        }
                     }
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(smem_u32(&bars->full[s]), IX_B_BYTES);
+                        mbar_arrive_expect_tx(smem_u32(&bars->full[s]), IX_B_BYTES + (bulk ? IX_BN * 4 : 0));
                         tma_load_2d(sB + s * IX_B_BYTES, &a.tm_k, 0, (int32_t)kr0, smem_u32(&bars->full[s]));
+                        if (bulk) bulk_load(smem_u32(scs), a.k_scale + kr0, IX_BN * 4, smem_u32(&bars->full[s]));
                     }
                     last_issued[s] = g;
                     __syncwarp();
@@ -211,14 +322,18 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
         const bool in_range = a.mode != 1 || (t >= a.row_begin && t < a.row_begin + a.row_count);
         const bool take_all = pos + 1 <= a.k;
         // radix state
-        int level = 0, sh = 31, P = 0;
-        uint32_t need = (uint32_t)a.k;
+        int level = 0;
+        RowSel rs;
+        rs.sh = 31;
+        rs.P = 0;
+        rs.need = (uint32_t)a.k;
+        rs.taken = 0;
+        rs.cnt = 0;
+        rs.take_all = take_all;
         bool resolved = !has_row || take_all;
         uint32_t* myhist = hist + row;  // bin b at myhist[b * IX_BM]
         int32_t* out = (a.mode == 0 && has_row) ? a.idx + t * a.ld_idx : nullptr;
         float* srow_out = (a.mode == 1 && has_row && in_range) ? a.scores + (t - a.row_begin) * a.ld_scores : nullptr;
-        int cnt = 0;
-        uint32_t taken = 0;
         for (int i = 0; i < 256; ++i) myhist[i * IX_BM] = 0;
 
         uint32_t g = 0;
@@ -233,52 +348,16 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
                 const float* scs = sc_s + s * IX_BN;
                 const int64_t s_tile = (int64_t)tile * IX_BN;
                 const bool active = ok && has_row && !(kind == SW_HIST && resolved);
-#pragma unroll 1
-                for (int ch = 0; ch < IX_BN / 32; ++ch) {
-                    uint32_t v[32];
-                    if (ok) {
-                        tmem_ld32(tmem + ((quad * 32) << 16) + ab * IX_BN + ch * 32, v);
-                        tmem_wait_ld();
-                    }
-                    if (!active) continue;
-                    const int64_t sbase = s_tile + ch * 32;
-                    if (sbase > pos) continue;
-                    const int lim = (int)min((int64_t)31, pos - sbase);  // columns 0..lim are causal
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (i > lim) break;
-                        const float x = __fmul_rn(__fmul_rn(__uint_as_float(v[i]), scs[ch * 32 + i]), srow);
-                        int kb = max(__float_as_int(x), 0);
-                        kb = min(kb, 0x7F800000);
-                        const int32_t sidx = (int32_t)(sbase + i);
-                        if (kind == SW_HIST) {
-                            if (lvl == 1) {
-                                atomicAdd(&myhist[((uint32_t)kb + 0x7FFFFFu) >> 23 << 7], 1u);
-                            } else {
-                                const int xk = kb - 1;
-                                if ((xk >> sh) == P) {
-                                    const uint32_t d = lvl == 2 ? ((uint32_t)xk >> 15) & 255u
-                                                     : lvl == 3 ? ((uint32_t)xk >> 7) & 255u
-                                                                : (uint32_t)xk & 127u;
-                                    atomicAdd(&myhist[d << 7], 1u);
-                                }
-                            }
-                        } else if (kind == SW_EMIT) {
-                            bool e = take_all;
-                            if (!e) {
-                                const int hi = (kb - 1) >> sh;
-                                if (hi > P) e = true;
-                                else if (hi == P && taken < need) { e = true; ++taken; }
-                            }
-                            if (e) {
-                                if (cnt < a.k) out[cnt] = sidx;
-                                ++cnt;
-                            }
-                        } else if (kind == SW_SCORES) {
-                            if (srow_out) srow_out[sidx] = __int_as_float(kb);
-                        }
-                    }
-                }
+                const uint32_t taddr = tmem + ((quad * 32) << 16) + ab * IX_BN;
+                if (kind == SW_HIST && lvl == 1)
+                    ep_tile<1>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
+                else if (kind == SW_HIST)
+                    ep_tile<4>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, lvl == 2 ? 15 : lvl == 3 ? 7 : 0,
+                               lvl == 4 ? 127u : 255u, out, a.k, srow_out);
+                else if (kind == SW_EMIT)
+                    ep_tile<2>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
+                else
+                    ep_tile<3>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -294,16 +373,16 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
                     const int top = lvl == 4 ? 127 : 255;
                     for (int bb = top; bb >= 0; --bb) {
                         const uint32_t c = myhist[bb * IX_BM];
-                        if (cum + c >= need) { bsel = bb; break; }
+                        if (cum + c >= rs.need) { bsel = bb; break; }
                         cum += c;
                     }
                     const uint32_t in_bin = myhist[bsel * IX_BM];
-                    need -= cum;
-                    if (lvl == 1) { P = bsel - 1; sh = 23; }
-                    else if (lvl == 2) { P = (P << 8) | bsel; sh = 15; }
-                    else if (lvl == 3) { P = (P << 8) | bsel; sh = 7; }
-                    else { P = (P << 7) | bsel; sh = 0; }
-                    resolved = in_bin == need || P == -1 || lvl == 4;
+                    rs.need -= cum;
+                    if (lvl == 1) { rs.P = bsel - 1; rs.sh = 23; }
+                    else if (lvl == 2) { rs.P = (rs.P << 8) | bsel; rs.sh = 15; }
+                    else if (lvl == 3) { rs.P = (rs.P << 8) | bsel; rs.sh = 7; }
+                    else { rs.P = (rs.P << 7) | bsel; rs.sh = 0; }
+                    resolved = in_bin == rs.need || rs.P == -1 || lvl == 4;
                 }
                 level = lvl;
                 for (int i = 0; i < 256; ++i) myhist[i * IX_BM] = 0;
@@ -325,11 +404,11 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
         if (a.mode == 0 && has_row) {
             if (first_kind == SW_STOP) {  // every row of the block keeps its whole prefix
                 for (int64_t s = 0; s <= pos; ++s) out[s] = (int32_t)s;
-                cnt = (int)(pos + 1);
+                rs.cnt = (int)(pos + 1);
             }
             const int expect = (int)min((int64_t)a.k, pos + 1);
-            if (cnt != expect && !*abort) report(st, DSA_ERR_INDEX, -2000000 - t);
-            for (int s = min(cnt, a.k); s < a.k; ++s) out[s] = -1;
+            if (rs.cnt != expect && !*abort) report(st, DSA_ERR_INDEX, -2000000 - t);
+            for (int s = min(rs.cnt, a.k); s < a.k; ++s) out[s] = -1;
         }
     }
     tc_fence_before();

@@ -50,14 +50,16 @@ _lib.dsa_index_scores.argtypes = [_S, _IA, _I64, _I64, _P, _I64, _P, _SZ, _P]
 _lib.dsa_topk.argtypes = [_S, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_sparse_attn.argtypes = [_S, _AA, _P, _I64, _I32, _P, _SZ, _P]
 _lib.dsa_forward.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P]
+_lib.dsa_select.argtypes = [_S, _IA, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_sync_status.argtypes = [_P, _P, ctypes.POINTER(_I64)]
 _lib.dsa_selftest_wait_timeout.argtypes = [_P, _SZ, _I64, _P]
 for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+           "dsa_select",
            "dsa_sync_status", "dsa_selftest_wait_timeout"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk",
-            "dsa_sparse_attn", "dsa_forward", "dsa_sync_status", "dsa_selftest_wait_timeout")
+            "dsa_sparse_attn", "dsa_forward", "dsa_select", "dsa_sync_status", "dsa_selftest_wait_timeout")
 
 
 class DsaError(RuntimeError):
@@ -175,6 +177,11 @@ def dsa_forward(seqs, ia, aa, k, idx_out, ws):
     _check(_lib.dsa_forward(ctypes.byref(seqs.c), ctypes.byref(ia), ctypes.byref(aa), k, _ptr(idx_out),
                             idx_out.stride(0) if idx_out is not None else 0, _ptr(ws), ws.numel(), _stream()),
            "dsa_forward")
+
+
+def dsa_select(seqs, ia, k, idx, ws):
+    _check(_lib.dsa_select(ctypes.byref(seqs.c), ctypes.byref(ia), k, _ptr(idx), idx.stride(0), _ptr(ws), ws.numel(),
+                           _stream()), "dsa_select")
 
 
 def dsa_sync_status(ws):
