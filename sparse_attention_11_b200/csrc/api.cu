@@ -239,12 +239,10 @@ int run_attn(const dsa_seqs* s, const dsa_attn_args* aa, const int32_t* idx, int
         a.k_sel = k_sel;
         a.v_separate = attn_v_separate(aa) ? 1 : 0;
         a.st = h;
-        const uint64_t rows = (uint64_t)(s->total_k > 0 ? s->total_k : 1);
-        if (!make_map_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, aa->k, 576, rows, (uint64_t)aa->k_stride * 2, 64, 1))
-            return DSA_ERR_CUDA;
-        if (a.v_separate &&
-            !make_map_2d(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, aa->v, 512, rows, (uint64_t)aa->v_stride * 2, 64, 1))
-            return DSA_ERR_CUDA;
+        a.k = (const __nv_bfloat16*)aa->k;
+        a.k_stride = aa->k_stride;
+        a.v = (const __nv_bfloat16*)aa->v;
+        a.v_stride = aa->v_stride;
         if (!launch_attn_tc(a, st)) return DSA_ERR_CUDA;
         return cuda_status();
     }

@@ -14,63 +14,78 @@
 // When V is the latent part of K (V = K[:, :512]) each CTA's V columns are
 // the first 256 of its own K columns, so every gathered byte is used once.
 //
-// Softmax split: per 64-key tile each CTA holds a partial S for all 128 heads
-// and all 64 keys.  Rank r finishes the scores of keys [32r, 32r+32) for all
-// heads: it sends the other 32 partial columns to its peer and receives the
-// peer's partials of its own 32 keys (st.async into the peer's shared memory,
-// counted on the peer's mbarrier).  Both CTAs use the same running maximum:
-// the sum of the two partial maxima of the tile, an upper bound of the true
-// maximum that both can form from the exchanged data, with lazy rescaling
-// (moved only when it grows by more than 2^8).  Each CTA then computes bf16
-// probabilities for its 32 keys, sends them to the peer, and accumulates its
-// half of O over all 64 keys.  The row sums are combined once at the end.
+// Softmax split.  Per 64-key tile each CTA holds a partial S for all 128
+// heads and all 64 keys.  Rank r finishes keys [32r, 32r+32): it sends the
+// other 32 partial columns to its peer and receives the peer's partials of
+// its own keys (st.async into the peer's shared memory, byte-counted on the
+// peer's mbarrier).  Both CTAs use the same running maximum: the sum of the
+// two partial maxima of the tile, an upper bound of the true maximum that
+// both form from the exchanged data, with lazy rescaling (moved only when it
+// grows by more than 2^8).  Each CTA writes the bf16 probabilities of its
+// keys into its own P tile and into the peer's, so both hold the full
+// 128 x 64 P (the A operand of O += P V, in shared memory).  Row sums are
+// combined once at the end.
 //
-// Tensor memory per CTA (512 columns): O [0,256)  S [256,320)  P [320,352)
-// Q [352, 352 + 32 * blocks).  Q and P are the A operands, read from TMEM
-// (tcgen05.mma ... [a_tmem]); K/V tiles are B operands in shared memory,
-// gathered by TMA tile::gather4 (4 rows x 64 columns per instruction, 128-byte
-// swizzle) straight from the KV rows named by the index list.
+// Pipelining.  The softmax warps run stage A of tile j+1 (read S, send the
+// partial) before stage B of tile j (combine, probabilities, write P), so each
+// exchange has a whole stage to land; the MMA warp issues S(t) then PV(t-2)
+// (PV(t-1) with only two K/V stages).
+// P tiles are double-buffered and released by a tcgen05.commit that arrives
+// on the p_free barrier of both CTAs (PV(t) done in both), so stage B waits
+// for PV(t-2), and for PV(t-1) only when the running maximum moves.
 //
-// Warps: 0 gather producer, 1 MMA issuer (+TMEM owner), 2..5 softmax /
-// exchange / epilogue (thread <-> head, the TMEM lane).
+// Gathers: two producer warps copy the selected rows with 16-byte cp.async,
+// 4 rows x 128 bytes per warp instruction, into the 128-byte-swizzled tile
+// layout the MMA reads (row r's 16-byte chunk c at chunk c ^ (r & 7)).
+//
+// Tensor memory per CTA: O [0,256)  S [256,320)  Q [320, 320 + 32 * blocks).
+// Warps: 0-1 producers, 2 MMA issuer (+TMEM owner), 3-6 softmax / exchange /
+// epilogue (thread <-> head, the TMEM lane).
 #include "dsa_kernels.h"
 
 namespace dsa {
 
-constexpr int AT_N = 64;                            // keys per tile
-constexpr uint32_t AT_BLK = AT_N * 128;             // one 64-column block of a tile
-constexpr uint32_t AT_KST = 5 * AT_BLK;             // K part of a stage (max 5 blocks)
-constexpr uint32_t AT_VST = 4 * AT_BLK;             // V part (separate V only)
-constexpr uint32_t AT_SX_PITCH = 144;               // 32 fp32 partials + partial max + pad
-constexpr uint32_t AT_PX_PITCH = 80;                // 32 bf16 probabilities + pad
-constexpr uint32_t AT_SX_BYTES = 128 * 9 * 16;      // bytes counted per tile
-constexpr uint32_t AT_PX_BYTES = 128 * 4 * 16;
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_P = 320, TM_Q = 352;
+constexpr int AT_N = 64;                           // keys per tile
+constexpr uint32_t AT_BLK = AT_N * 128;            // one 64-column block of a tile
+constexpr uint32_t AT_KST = 5 * AT_BLK;            // K part of a stage (max 5 blocks)
+constexpr uint32_t AT_VST = 4 * AT_BLK;            // V part (separate V only)
+constexpr uint32_t AT_TILE128 = 128 * 128;         // a 128-row x 128-byte swizzled tile
+constexpr uint32_t AT_SX_BYTES = 128 * 128 + 128 * 4;  // partial scores + partial maxima
+constexpr uint32_t AT_PX_BYTES = 128 * 64;         // the peer's half of P
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320;
+constexpr int AT_THREADS = 224;
 
 template <int NST, bool VSEP>
 struct AtLayout {
     static constexpr uint32_t STAGE = AT_KST + (VSEP ? AT_VST : 0);
-    static constexpr uint32_t OFF_SX = NST * STAGE;                   // [2][128][144]
-    static constexpr uint32_t OFF_PX = OFF_SX + 2 * 128 * AT_SX_PITCH;  // [2][128][80]
-    static constexpr uint32_t OFF_LX = OFF_PX + 2 * 128 * AT_PX_PITCH;  // [128] fp32
+    static constexpr uint32_t OFF_P = NST * STAGE;            // [2] P tiles
+    static constexpr uint32_t OFF_SX = OFF_P + 2 * AT_TILE128;  // [2] partial-score tiles
+    static constexpr uint32_t OFF_PM = OFF_SX + 2 * AT_TILE128; // [2][128] partial maxima
+    static constexpr uint32_t OFF_LX = OFF_PM + 2 * 512;        // [128] peer row sums
     static constexpr uint32_t OFF_BAR = OFF_LX + 512;
-    static constexpr uint32_t SMEM = OFF_BAR + 512 + 1024;
+    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 
 struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
-    uint64_t s_full, s_empty, p_full, p_free, q_full, o_full;
-    uint64_t sx_full[2], px_full[2], lx_full;  // filled by the peer (st.async, byte-counted)
-    uint64_t sx_free[2], px_free[2];           // the peer consumed what this CTA sent
-    uint64_t drain;
+    uint64_t s_full, s_empty, q_full, o_full;
+    uint64_t p_full[2];   // 4 local warps + the peer's half of P (bytes)
+    uint64_t p_free[2];   // PV done in both CTAs (multicast commit)
+    uint64_t sx_full[2];  // the peer's partial scores (bytes)
+    uint64_t sx_free[2];  // the peer consumed the partials this CTA sent
+    uint64_t lx_full, drain;
     uint32_t tmem_base;
     int abort;
     int max_slot;
 };
+static_assert(sizeof(AtBars) <= 256, "barrier block");
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 
 template <int NST, bool VSEP>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__ AttnTcArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ AttnTcArgs a) {
     using Lay = AtLayout<NST, VSEP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -86,41 +101,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         if (threadIdx.x == 0 && rank == 0) report(st, DSA_ERR_INDEX, t);
         return;
     }
-    const int nb = rank ? 5 : 4;           // 64-column blocks of K held here
-    const int col0 = rank ? 256 : 0;       // first K column
-    const int dv0 = rank ? 256 : 0;        // first output column
+    const int nb = rank ? 5 : 4;      // 64-column blocks of K held here
+    const int col0 = rank ? 256 : 0;  // first K column
+    const int dv0 = rank ? 256 : 0;   // first output column
     const int32_t* irow = a.idx + t * a.ld_idx;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
-            mbar_init(smem_u32(&bars->full[i]), 1);
+            mbar_init(smem_u32(&bars->full[i]), 64);
             mbar_init(smem_u32(&bars->empty[i]), 1);
         }
         mbar_init(smem_u32(&bars->s_full), 1);
         mbar_init(smem_u32(&bars->s_empty), 4);
-        mbar_init(smem_u32(&bars->p_full), 4);
-        mbar_init(smem_u32(&bars->p_free), 1);
         mbar_init(smem_u32(&bars->q_full), 4);
         mbar_init(smem_u32(&bars->o_full), 1);
         for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bars->p_full[i]), 4);
+            mbar_init(smem_u32(&bars->p_free[i]), 2);
             mbar_init(smem_u32(&bars->sx_full[i]), 1);
-            mbar_init(smem_u32(&bars->px_full[i]), 1);
             mbar_init(smem_u32(&bars->sx_free[i]), 4);
-            mbar_init(smem_u32(&bars->px_free[i]), 4);
         }
         mbar_init(smem_u32(&bars->lx_full), 1);
         mbar_init(smem_u32(&bars->drain), 1);
-        // arm the byte-counted barriers for their first phase
+        // byte counts of the first phase of every peer-filled barrier
         for (int i = 0; i < 2; ++i) {
+            mbar_expect_tx(smem_u32(&bars->p_full[i]), AT_PX_BYTES);
             mbar_arrive_expect_tx(smem_u32(&bars->sx_full[i]), AT_SX_BYTES);
-            mbar_arrive_expect_tx(smem_u32(&bars->px_full[i]), AT_PX_BYTES);
         }
         mbar_arrive_expect_tx(smem_u32(&bars->lx_full), 128 * 4);
         bars->abort = 0;
         bars->max_slot = -1;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    if (warp == 2) tmem_alloc(smem_u32(&bars->tmem_base), 512);
     __syncthreads();
     // number of 64-slot tiles: up to the last valid slot of the index row
     {
@@ -137,76 +150,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
     const int n_tiles = (bars->max_slot + AT_N) / AT_N;
 
     const uint32_t s_stage0 = smem_u32(smem);
-    if (warp == 0) {
-        // ================= gather producer =================
-        if (lane == 0) {
-            tma_prefetch_desc(&a.tm_k);
-            if (VSEP) tma_prefetch_desc(&a.tm_v);
+    const uint32_t s_p0 = smem_u32(smem + Lay::OFF_P);
+    if (warp < 2) {
+        // ================= gather producers (64 threads) =================
+        const __nv_bfloat16* kbase = a.k;
+        const __nv_bfloat16* vbase = a.v;
+        const int key_in_warp = (int)(lane >> 3), chunk = (int)(lane & 7);
+        int32_t nxt = -1;
+        if (n_tiles > 0) {
+            const int slot = (int)(warp * 32 + lane);
+            nxt = slot < a.k_sel ? __ldg(irow + slot) : -1;
         }
-        uint32_t last_issued[NST];
-        for (int i = 0; i < NST; ++i) last_issued[i] = 0xFFFFFFFFu;
-        int32_t nxt[4];
-        auto load_rows = [&](int j, int32_t (&rw)[4]) {
-            if (lane < 16) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int slot = j * AT_N + lane * 4 + i;
-                    rw[i] = slot < a.k_sel ? __ldg(irow + slot) : -1;
-                }
-            }
-        };
-        if (n_tiles > 0) load_rows(0, nxt);
         for (int j = 0; j < n_tiles; ++j) {
             const uint32_t s = j % NST;
-            int32_t rows[4];
+            int32_t v = nxt;
+            if (j + 1 < n_tiles) {
+                const int slot = (j + 1) * AT_N + (int)(warp * 32 + lane);
+                nxt = slot < a.k_sel ? __ldg(irow + slot) : -1;
+            }
+            if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
+            const int64_t row = ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0);
+            if (!wait_warp(smem_u32(&bars->empty[s]), ((j / NST) & 1) ^ 1, abort, st, 0x2101)) break;
+            const uint32_t kst = s_stage0 + s * Lay::STAGE;
+#pragma unroll 1
+            for (int q = 0; q < 8; ++q) {
+                const int key = (int)(warp * 32) + 4 * q + key_in_warp;  // key of the tile
+                const int64_t r = __shfl_sync(0xffffffffu, row, 4 * q + key_in_warp);
+                const __nv_bfloat16* src = kbase + r * a.k_stride + col0 + chunk * 8;
+                const uint32_t dst = kst + swz(key, chunk);
+                for (int kb = 0; kb < nb; ++kb) cp_async16(dst + kb * AT_BLK, src + kb * 64);
+                if (VSEP) {
+                    const __nv_bfloat16* vs = vbase + r * a.v_stride + dv0 + chunk * 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rows[i] = nxt[i];
-            if (j + 1 < n_tiles) load_rows(j + 1, nxt);
-            if (lane < 16) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int32_t v = rows[i];
-                    if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
-                    rows[i] = (int32_t)(ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0));
+                    for (int vb = 0; vb < 4; ++vb) cp_async16(dst + AT_KST + vb * AT_BLK, vs + vb * 64);
                 }
             }
-            if (!wait_warp(smem_u32(&bars->empty[s]), ((j / NST) & 1) ^ 1, abort, st, 0x2101)) break;
-            if (lane == 0)
-                mbar_arrive_expect_tx(smem_u32(&bars->full[s]), nb * AT_BLK + (VSEP ? AT_VST : 0));
-            __syncwarp();
-            if (lane < 16) {
-                const uint32_t kst = s_stage0 + s * Lay::STAGE;
-                for (int kb = 0; kb < nb; ++kb)
-                    tma_gather4(kst + kb * AT_BLK + lane * 512, &a.tm_k, col0 + kb * 64, rows[0], rows[1], rows[2], rows[3],
-                                smem_u32(&bars->full[s]));
-                if (VSEP)
-                    for (int vb = 0; vb < 4; ++vb)
-                        tma_gather4(kst + AT_KST + vb * AT_BLK + lane * 512, &a.tm_v, dv0 + vb * 64, rows[0], rows[1], rows[2],
-                                    rows[3], smem_u32(&bars->full[s]));
-            }
-            last_issued[s] = j;
-            __syncwarp();
+            cp_async_arrive(smem_u32(&bars->full[s]));
         }
-        if (*abort && lane == 0)
-            for (int s = 0; s < NST; ++s)
-                if (last_issued[s] != 0xFFFFFFFFu)
-                    mbar_wait(smem_u32(&bars->full[s]), (last_issued[s] / NST) & 1, nullptr, st, 0x2102, 1ll << 28);
-    } else if (warp == 1) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 2) {
         // ================= MMA issuer =================
         constexpr uint32_t idesc_s = idesc_make(1, 1, false, 128, AT_N);
         constexpr uint32_t idesc_pv = idesc_make(1, 1, true, 128, 256);
+        // PV(t - kLag) follows S(t); S(t) reuses the stage PV(t - NST) frees,
+        // so the lag must stay below the stage count.
+        constexpr int kLag = NST >= 3 ? 2 : 1;
         bool ok = n_tiles > 0 && wait_warp(smem_u32(&bars->q_full), 0, abort, st, 0x2201);
-        auto issue_pv = [&](int jj) -> bool {
-            if (!wait_warp(smem_u32(&bars->p_full), jj & 1, abort, st, 0x2202)) return false;
+        auto issue_pv = [&](int u) -> bool {
+            const uint32_t b = u & 1;
+            if (!wait_warp(smem_u32(&bars->p_full[b]), (u >> 1) & 1, abort, st, 0x2202)) return false;
+            fence_proxy_async();
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t vbase = s_stage0 + (jj % NST) * Lay::STAGE + (VSEP ? AT_KST : 0);
+                if (u + 2 < n_tiles) mbar_expect_tx(smem_u32(&bars->p_full[b]), AT_PX_BYTES);
+                const uint32_t vb = s_stage0 + (u % NST) * Lay::STAGE + (VSEP ? AT_KST : 0);
+                const uint32_t pb = s_p0 + b * AT_TILE128;
 #pragma unroll
                 for (int ks = 0; ks < AT_N / 16; ++ks)
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_P + ks * 8, sdesc_sw128(vbase + ks * 2048, AT_BLK, 1024), idesc_pv,
-                                (jj > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(smem_u32(&bars->empty[jj % NST]));
-                mma_commit(smem_u32(&bars->p_free));
+                    mma_bf16_ss(tmem + TM_O, sdesc_sw128(pb + ks * 32, 16, 1024), sdesc_sw128(vb + ks * 2048, AT_BLK, 1024),
+                                idesc_pv, (u > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(smem_u32(&bars->empty[u % NST]));
+                mma_commit_mc(smem_u32(&bars->p_free[b]), (uint16_t)3);
             }
             __syncwarp();
             return true;
@@ -214,6 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         for (int j = 0; ok && j < n_tiles; ++j) {
             const uint32_t s = j % NST;
             if (!wait_warp(smem_u32(&bars->full[s]), (j / NST) & 1, abort, st, 0x2203)) { ok = false; break; }
+            fence_proxy_async();
             if (!wait_warp(smem_u32(&bars->s_empty), (j & 1) ^ 1, abort, st, 0x2204)) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) {
@@ -226,11 +231,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
                 mma_commit(smem_u32(&bars->s_full));
             }
             __syncwarp();
-            if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            if (j >= kLag && !issue_pv(j - kLag)) { ok = false; break; }
         }
-        if (ok && n_tiles > 0 && issue_pv(n_tiles - 1)) {
-            if (lane == 0) mma_commit(smem_u32(&bars->o_full));
-        }
+        for (int u = n_tiles >= kLag ? n_tiles - kLag : 0; ok && u < n_tiles; ++u)
+            if (!issue_pv(u)) ok = false;
+        if (ok && n_tiles > 0 && lane == 0) mma_commit(smem_u32(&bars->o_full));
         if (*abort && lane == 0) {
             mma_commit(smem_u32(&bars->drain));
             mbar_wait(smem_u32(&bars->drain), 0, nullptr, st, 0x2205, 1ll << 28);
@@ -240,22 +245,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
         const uint32_t quad = warp & 3;
         const int h = (int)(quad * 32 + lane);
         const uint32_t lane_off = (quad * 32) << 16;
-        const int kh = (int)rank;             // this CTA's key half of every tile
+        const int kh = (int)rank;  // this CTA's key half of every tile
         uint8_t* sx = smem + Lay::OFF_SX;
-        uint8_t* px = smem + Lay::OFF_PX;
-        float* lx = (float*)(smem + Lay::OFF_LX);
+        const float* pmx = (const float*)(smem + Lay::OFF_PM);
+        const float* lx = (const float*)(smem + Lay::OFF_LX);
         const uint32_t peer_sx = mapa(smem_u32(sx), peer);
-        const uint32_t peer_px = mapa(smem_u32(px), peer);
-        const uint32_t peer_lx = mapa(smem_u32(lx), peer);
-        // peer barrier addresses of buffer b are base + 8 b (same layout in both CTAs)
+        const uint32_t peer_pm = mapa(smem_u32(smem + Lay::OFF_PM), peer);
+        const uint32_t peer_p = mapa(s_p0, peer);
+        const uint32_t peer_lx = mapa(smem_u32(smem + Lay::OFF_LX), peer);
         const uint32_t peer_sx_full0 = mapa(smem_u32(&bars->sx_full[0]), peer);
-        const uint32_t peer_px_full0 = mapa(smem_u32(&bars->px_full[0]), peer);
         const uint32_t peer_sx_free0 = mapa(smem_u32(&bars->sx_free[0]), peer);
-        const uint32_t peer_px_free0 = mapa(smem_u32(&bars->px_free[0]), peer);
-        const uint32_t my_sx_full0 = smem_u32(&bars->sx_full[0]), my_px_full0 = smem_u32(&bars->px_full[0]);
-        const uint32_t my_sx_free0 = smem_u32(&bars->sx_free[0]), my_px_free0 = smem_u32(&bars->px_free[0]);
+        const uint32_t peer_p_full0 = mapa(smem_u32(&bars->p_full[0]), peer);
         const uint32_t peer_lx_full = mapa(smem_u32(&bars->lx_full), peer);
-        const bool arm_thread = threadIdx.x == 64;
+        const uint32_t my_sx_full0 = smem_u32(&bars->sx_full[0]), my_sx_free0 = smem_u32(&bars->sx_free[0]);
+        const uint32_t my_p_full0 = smem_u32(&bars->p_full[0]), my_p_free0 = smem_u32(&bars->p_free[0]);
+        const bool arm_thread = threadIdx.x == 96;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
@@ -276,80 +280,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
         }
-        int32_t nv0 = -1, nv1 = -1;
+        // per-tile data carried from stage A to stage B
+        float mine_cur[32], mine_nxt[32];
+        float pm_cur = -INFINITY, pm_nxt = -INFINITY;
+        uint32_t msk_cur = 0, msk_nxt = 0;
+        int32_t iv0 = -1, iv1 = -1;  // slots of the next tile to read
         if (n_tiles > 0) {
-            nv0 = lane < a.k_sel ? __ldg(irow + lane) : -1;
-            nv1 = lane + 32 < a.k_sel ? __ldg(irow + lane + 32) : -1;
+            iv0 = (int)lane < a.k_sel ? __ldg(irow + lane) : -1;
+            iv1 = (int)lane + 32 < a.k_sel ? __ldg(irow + lane + 32) : -1;
         }
-        for (int j = 0; ok && j < n_tiles; ++j) {
-            const uint32_t b = j & 1, ph = (j >> 1) & 1;
-            const int32_t v0 = nv0, v1 = nv1;
-            if (j + 1 < n_tiles) {  // prefetch the next tile's slots
-                const int sl0 = (j + 1) * AT_N + lane, sl1 = sl0 + 32;
-                nv0 = sl0 < a.k_sel ? __ldg(irow + sl0) : -1;
-                nv1 = sl1 < a.k_sel ? __ldg(irow + sl1) : -1;
+        // Stage A of tile u: read S, partial max, send the peer's half.
+        auto stage_a = [&](int u) -> bool {
+            const uint32_t b = u & 1, ph = (u >> 1) & 1;
+            const uint32_t mlo = __ballot_sync(0xffffffffu, iv0 >= 0 && iv0 < ri.seqlen_k);
+            const uint32_t mhi = __ballot_sync(0xffffffffu, iv1 >= 0 && iv1 < ri.seqlen_k);
+            if (u + 1 < n_tiles) {  // prefetch the following tile's slots
+                const int sl0 = (u + 1) * AT_N + (int)lane, sl1 = sl0 + 32;
+                iv0 = sl0 < a.k_sel ? __ldg(irow + sl0) : -1;
+                iv1 = sl1 < a.k_sel ? __ldg(irow + sl1) : -1;
             }
-            const uint32_t mlo = __ballot_sync(0xffffffffu, v0 >= 0 && v0 < ri.seqlen_k);
-            const uint32_t mhi = __ballot_sync(0xffffffffu, v1 >= 0 && v1 < ri.seqlen_k);
-            const uint32_t mine = kh ? mhi : mlo;      // validity of this CTA's 32 keys
-            if (!wait_warp(smem_u32(&bars->s_full), j & 1, abort, st, 0x2301)) { ok = false; break; }
+            if (!wait_warp(smem_u32(&bars->s_full), u & 1, abort, st, 0x2301)) return false;
             tc_fence_after();
-            float sa[64];
-            {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_off + TM_S, r0);
-                tmem_ld32(tmem + lane_off + TM_S + 32, r1);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    sa[i] = __uint_as_float(r0[i]);
-                    sa[32 + i] = __uint_as_float(r1[i]);
-                }
-            }
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tmem + lane_off + TM_S, r0);
+            tmem_ld32(tmem + lane_off + TM_S + 32, r1);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
-            // partial maximum over the tile's valid keys
             float pm = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                if ((mlo >> i) & 1u) pm = fmaxf(pm, sa[i]);
-                if ((mhi >> i) & 1u) pm = fmaxf(pm, sa[32 + i]);
+                if ((mlo >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r0[i]));
+                if ((mhi >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r1[i]));
             }
-            // send the peer's 32 partial columns and the partial max
-            if (!wait_warp_cluster(my_sx_free0 + 8 * b, ph ^ 1, abort, st, 0x2302)) { ok = false; break; }
-            {
-                const uint32_t dst = peer_sx + b * (128 * AT_SX_PITCH) + h * AT_SX_PITCH;
+            if (!wait_warp(my_sx_free0 + 8 * b, ph ^ 1, abort, st, 0x2302)) return false;
+            const uint32_t dst = peer_sx + b * AT_TILE128;
+            const uint32_t bar = peer_sx_full0 + 8 * b;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    // the peer's keys: [32, 64) for rank 0, [0, 32) for rank 1
-                    uint32_t w[4];
+            for (int c = 0; c < 8; ++c) {  // the peer's keys: [32,64) for rank 0, [0,32) for rank 1
+                uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) w[e] = __float_as_uint(kh ? sa[4 * c + e] : sa[32 + 4 * c + e]);
-                    st_async_v4(dst + c * 16, w[0], w[1], w[2], w[3], peer_sx_full0 + 8 * b);
-                }
-                st_async_v4(dst + 128, __float_as_uint(pm), 0u, 0u, 0u, peer_sx_full0 + 8 * b);
+                for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
+                st_async_v4(dst + swz(h, c), w[0], w[1], w[2], w[3], bar);
             }
-            // receive the peer's partials of this CTA's 32 keys
-            if (!wait_warp_cluster(my_sx_full0 + 8 * b, ph, abort, st, 0x2303)) { ok = false; break; }
-            if (arm_thread && j + 2 < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * b, AT_SX_BYTES);
+            st_async_b32(peer_pm + b * 512 + h * 4, __float_as_uint(pm), bar);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mine_nxt[i] = __uint_as_float(kh ? r1[i] : r0[i]);
+            pm_nxt = pm;
+            msk_nxt = kh ? mhi : mlo;
+            return true;
+        };
+        // Stage B of tile u: combine, probabilities, write both copies of P.
+        auto stage_b = [&](int u) -> bool {
+            const uint32_t b = u & 1, ph = (u >> 1) & 1;
+            if (!wait_warp(my_sx_full0 + 8 * b, ph, abort, st, 0x2303)) return false;
+            if (arm_thread && u + 2 < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * b, AT_SX_BYTES);
             float s32[32];
-            float pm_peer;
             {
-                const float4* src = (const float4*)(sx + b * (128 * AT_SX_PITCH) + h * AT_SX_PITCH);
+                const uint8_t* rowp = sx + b * AT_TILE128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const float4 v = src[c];
-                    const float pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) s32[4 * c + e] = (kh ? sa[32 + 4 * c + e] : sa[4 * c + e]) + pv[e];
+                    const float4 v = *(const float4*)(rowp + swz(h, c));
+                    s32[4 * c] = mine_cur[4 * c] + v.x;
+                    s32[4 * c + 1] = mine_cur[4 * c + 1] + v.y;
+                    s32[4 * c + 2] = mine_cur[4 * c + 2] + v.z;
+                    s32[4 * c + 3] = mine_cur[4 * c + 3] + v.w;
                 }
-                pm_peer = src[8].x;
             }
+            const float pm_peer = pmx[b * 128 + h];
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * b);
             // shared running maximum (identical in both CTAs), lazy rescale
-            const float mb = (pm == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm + pm_peer) * a.scale_log2;
+            const float mb = (pm_cur == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm_cur + pm_peer) * a.scale_log2;
             float alpha = 1.f;
             if (mb > m_used + 8.0f) {
                 alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mb);
@@ -358,28 +361,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
             }
             uint32_t pw[16];
             {
-                float rs = 0.f;
+                float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float p0 = ((mine >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
-                    const float p1 = ((mine >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
-                    rs += p0 + p1;
+                    const float p0 = ((msk_cur >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
+                    const float p1 = ((msk_cur >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
+                    rs0 += p0;
+                    rs1 += p1;
                     pw[i] = pack_bf16(p0, p1);
                 }
-                l += rs;
+                l += rs0 + rs1;
             }
-            // send this CTA's probabilities to the peer
-            if (!wait_warp_cluster(my_px_free0 + 8 * b, ph ^ 1, abort, st, 0x2304)) { ok = false; break; }
+            // P tile b is free once PV(u-2) is done in both CTAs
+            if (!wait_warp(my_p_free0 + 8 * b, ph ^ 1, abort, st, 0x2304)) return false;
             {
-                const uint32_t dst = peer_px + b * (128 * AT_PX_PITCH) + h * AT_PX_PITCH;
+                uint8_t* prow = smem + Lay::OFF_P + b * AT_TILE128;
+                const uint32_t pdst = peer_p + b * AT_TILE128;
+                const uint32_t bar = peer_p_full0 + 8 * b;
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    st_async_v4(dst + c * 16, pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3], peer_px_full0 + 8 * b);
+                for (int q = 0; q < 4; ++q) {
+                    const int c = 4 * kh + q;
+                    *(uint4*)(prow + swz(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
+                    st_async_v4(pdst + swz(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
+                }
             }
-            // O rescale and this CTA's P half -> TMEM once the previous P.V is done
-            if (!wait_warp(smem_u32(&bars->p_free), (j & 1) ^ 1, abort, st, 0x2305)) { ok = false; break; }
-            tc_fence_after();
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // O may be rescaled only between PV(u-1) and PV(u)
+                const int w = u - 1;
+                if (!wait_warp(my_p_free0 + 8 * (w & 1), (w >> 1) & 1, abort, st, 0x2305)) return false;
+                tc_fence_after();
                 for (int c = 0; c < 8; ++c) {
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_off + TM_O + c * 32, r);
@@ -388,39 +398,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
                     tmem_st32(tmem + lane_off + TM_O + c * 32, r);
                 }
+                tmem_wait_st();
             }
-            tmem_st16(tmem + lane_off + TM_P + 16 * kh, pw);
-            // the peer's P half
-            if (!wait_warp_cluster(my_px_full0 + 8 * b, ph, abort, st, 0x2306)) { ok = false; break; }
-            if (arm_thread && j + 2 < n_tiles) mbar_arrive_expect_tx(my_px_full0 + 8 * b, AT_PX_BYTES);
-            {
-                uint32_t r[16];
-                const uint4* src = (const uint4*)(px + b * (128 * AT_PX_PITCH) + h * AT_PX_PITCH);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = src[c];
-                    r[4 * c] = v.x; r[4 * c + 1] = v.y; r[4 * c + 2] = v.z; r[4 * c + 3] = v.w;
-                }
-                tmem_st16(tmem + lane_off + TM_P + 16 * (1 - kh), r);
-            }
-            tmem_wait_st();
+            fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&bars->p_full));
-                mbar_arrive_remote(peer_px_free0 + 8 * b);
-            }
+            if (lane == 0) mbar_arrive(my_p_full0 + 8 * b);
+            return true;
+        };
+        if (n_tiles > 0) ok = stage_a(0);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mine_cur[i] = mine_nxt[i];
+            pm_cur = pm_nxt;
+            msk_cur = msk_nxt;
+            if (j + 1 < n_tiles && !stage_a(j + 1)) { ok = false; break; }
+            if (!stage_b(j)) { ok = false; break; }
         }
         // ---- row sums of both halves ----
         float l_tot = 0.f;
         if (ok && n_tiles > 0) {
             st_async_b32(peer_lx + h * 4, __float_as_uint(l), peer_lx_full);
-            if (wait_warp_cluster(smem_u32(&bars->lx_full), 0, abort, st, 0x2307)) l_tot = l + lx[h];
+            if (wait_warp(smem_u32(&bars->lx_full), 0, abort, st, 0x2306)) l_tot = l + lx[h];
             else ok = false;
         }
         // ---- epilogue: O / l -> bf16 ----
         __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0;
-        const bool have_o = ok && n_tiles > 0 && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2308);
+        const bool have_o = ok && n_tiles > 0 && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2307);
         if (have_o) tc_fence_after();
         const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
         for (int c = 0; c < 8; ++c) {
@@ -451,16 +455,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1) attn_tc_kern
     __syncwarp();
     cluster_sync();  // no DSMEM traffic may target a CTA that has exited
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
 template <int NST, bool VSEP>
 static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
     using Lay = AtLayout<NST, VSEP>;
+    static_assert(Lay::SMEM <= 232448, "shared memory budget");
     if (cudaFuncSetAttribute(attn_tc_kernel<NST, VSEP>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM) !=
         cudaSuccess)
         return false;
-    attn_tc_kernel<NST, VSEP><<<(unsigned)(2 * a.total_q), 192, Lay::SMEM, s>>>(a);
+    attn_tc_kernel<NST, VSEP><<<(unsigned)(2 * a.total_q), AT_THREADS, Lay::SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }
 

@@ -8,7 +8,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "../../include/dsa.h"
+#include "dsa.h"
 
 #define DSA_DEV __device__ __forceinline__
 
@@ -77,14 +77,27 @@ DSA_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;"
 DSA_DEV void mbar_arrive(uint32_t bar) {
     asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(bar) : "memory");
 }
+DSA_DEV void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// 16-byte asynchronous copy global -> shared (L2 only), and an arrive on `bar`
+// once every cp.async of this thread issued so far has landed (the arrival
+// is counted in the barrier's expected count).
+DSA_DEV void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"((uint64_t)src) : "memory");
+}
+DSA_DEV void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 DSA_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
 // Arrive on an mbarrier of another CTA of the cluster (cluster-space address
-// from mapa), releasing this thread's prior writes at cluster scope.
+// from mapa).  Used to hand a buffer back to the peer that fills it: this
+// thread's reads of the buffer are ordered before the arrive.
 DSA_DEV void mbar_arrive_remote(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 DSA_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
@@ -271,6 +284,14 @@ DSA_DEV void mma_fp8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_
     asm volatile(
         "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+// Arrive on the mbarrier at this shared-memory offset in every CTA of
+// `cta_mask` once every MMA issued so far by this thread has completed.
+DSA_DEV void mma_commit_mc(uint32_t bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(cta_mask)
         : "memory");
 }
 // Arrive on a CTA-local mbarrier once every MMA issued so far by this thread

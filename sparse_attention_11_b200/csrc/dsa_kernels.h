@@ -112,8 +112,10 @@ struct AttnTcArgs {
     int k_sel;
     int v_separate;         // 0: V = K[:, :512] (same rows); 1: own tensor
     StatusHdr* st;
-    CUtensorMap tm_k;       // K rows [total_k, 576], box 64x1, 128B swizzle
-    CUtensorMap tm_v;       // V rows [total_k, 512] (v_separate)
+    const __nv_bfloat16* k; // K rows [total_k, >= 576], row stride k_stride
+    int64_t k_stride;
+    const __nv_bfloat16* v; // V rows [total_k, >= 512] (v_separate)
+    int64_t v_stride;
 };
 bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s);
 
