@@ -108,7 +108,8 @@ typedef struct dsa_indexer_args {
  * {32,64,96,128} (exact fp32 SIMT kernel).  v may alias k (V = first dv
  * columns of each K row, as in MLA) by passing v = k and v_stride = k_stride.
  * BF16 requires 16-byte aligned q/k/v/out, k_stride and v_stride multiples of
- * 8 and q row strides multiples of 8. */
+ * 8, q row strides multiples of 8, and at most 2048 index slots per query
+ * (k_sel / k <= 2048); larger values return DSA_ERR_UNSUPPORTED. */
 typedef struct dsa_attn_args {
     int32_t dtype;          /* DSA_BF16 | DSA_F32 (q, k, v and out) */
     int32_t heads, dk, dv;

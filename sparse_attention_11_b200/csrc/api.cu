@@ -11,6 +11,7 @@ namespace {
 
 constexpr size_t kHdr = 256;
 constexpr int64_t kTcIndexerMinRows = 64;  // prefill-shaped query sets use the tensor-core indexer
+constexpr int32_t kTcAttnMaxSel = 2048;    // slots per query of the tensor-core attention
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -364,6 +365,7 @@ int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t
     if (!r) r = check_attn(seqs, aa);
     if (r) return r;
     if (k_sel < 0 || ld_idx < k_sel || (seqs->total_q && k_sel && !idx)) return DSA_ERR_INVALID_ARG;
+    if (attn_is_tc(aa) && k_sel > kTcAttnMaxSel) return DSA_ERR_UNSUPPORTED;
     r = check_ws(ws, ws_bytes, kHdr);
     if (r) return r;
     return run_attn(seqs, aa, idx, ld_idx, k_sel, hdr(ws), (cudaStream_t)stream);
@@ -406,6 +408,7 @@ int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn
     if (!r) r = check_attn(seqs, aa);
     if (r) return r;
     if (k < 1) return DSA_ERR_INVALID_ARG;
+    if (attn_is_tc(aa) && k > kTcAttnMaxSel) return DSA_ERR_UNSUPPORTED;
     if (idx_out && ld_idx < k) return DSA_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia));
     r = check_ws(ws, ws_bytes, L.total);

@@ -22,9 +22,9 @@
 // two partial maxima of the tile, an upper bound of the true maximum that
 // both form from the exchanged data, with lazy rescaling (moved only when it
 // grows by more than 2^8).  Each CTA writes the bf16 probabilities of its
-// keys into its own P tile and into the peer's, so both hold the full
-// 128 x 64 P (the A operand of O += P V, in shared memory).  Row sums are
-// combined once at the end.
+// keys into its own P tile and into the peer's (both with st.async), so both
+// hold the full 128 x 64 P (the A operand of O += P V, in shared memory).
+// Row sums are combined once at the end.
 //
 // Pipelining.  The softmax warps run stage A of tile j+1 (read S, send the
 // partial) before stage B of tile j (combine, probabilities, write P), so each
@@ -34,13 +34,17 @@
 // on the p_free barrier of both CTAs (PV(t) done in both), so stage B waits
 // for PV(t-2), and for PV(t-1) only when the running maximum moves.
 //
-// Gathers: two producer warps copy the selected rows with 16-byte cp.async,
-// 4 rows x 128 bytes per warp instruction, into the 128-byte-swizzled tile
-// layout the MMA reads (row r's 16-byte chunk c at chunk c ^ (r & 7)).
+// Gathers: seven producer warps copy the selected rows with 16-byte
+// cp.async, 4 rows x 128 bytes per warp instruction, into the
+// 128-byte-swizzled tile layout the MMA reads (row r's 16-byte chunk c at
+// chunk c ^ (r & 7)).  Gather throughput grows with the number of issuing
+// warps, so the producers are many and small (setmaxnreg moves their
+// registers to the softmax warps).
 //
 // Tensor memory per CTA: O [0,256)  S [256,320)  Q [320, 320 + 32 * blocks).
-// Warps: 0-1 producers, 2 MMA issuer (+TMEM owner), 3-6 softmax / exchange /
-// epilogue (thread <-> head, the TMEM lane).
+// Warps: 0-6 producers, 7 MMA issuer (+TMEM owner), 8-15 softmax / exchange /
+// epilogue: two warps per TMEM lane quadrant (thread <-> head), splitting
+// each tile's keys and O's columns.
 #include "dsa_kernels.h"
 
 namespace dsa {
@@ -53,7 +57,10 @@ constexpr uint32_t AT_TILE128 = 128 * 128;         // a 128-row x 128-byte swizz
 constexpr uint32_t AT_SX_BYTES = 128 * 128 + 128 * 4;  // partial scores + partial maxima
 constexpr uint32_t AT_PX_BYTES = 128 * 64;         // the peer's half of P
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320;
-constexpr int AT_THREADS = 224;
+constexpr int AT_THREADS = 512;  // 7 producer + 1 MMA + 8 softmax warps
+constexpr int AT_PRODUCERS = 7;
+constexpr int AT_MMA_WARP = 7;
+constexpr int AT_SOFT0 = 8;     // first softmax warp (a warpgroup boundary)
 
 template <int NST, bool VSEP>
 struct AtLayout {
@@ -61,20 +68,21 @@ struct AtLayout {
     static constexpr uint32_t OFF_P = NST * STAGE;            // [2] P tiles
     static constexpr uint32_t OFF_SX = OFF_P + 2 * AT_TILE128;  // [2] partial-score tiles
     static constexpr uint32_t OFF_PM = OFF_SX + 2 * AT_TILE128; // [2][128] partial maxima
-    static constexpr uint32_t OFF_LX = OFF_PM + 2 * 512;        // [128] peer row sums
-    static constexpr uint32_t OFF_BAR = OFF_LX + 512;
-    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+    static constexpr uint32_t OFF_LX = OFF_PM + 2 * 512;        // [2][128] this CTA's row-sum partials
+    static constexpr uint32_t OFF_VM = OFF_LX + 1024;            // [64] validity bits of 2048 slots
+    static constexpr uint32_t OFF_BAR = OFF_VM + 256;
+    static constexpr uint32_t SMEM = OFF_BAR + 256;
 };
 
 struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
     uint64_t s_full, s_empty, q_full, o_full;
-    uint64_t p_full[2];   // 4 local warps + the peer's half of P (bytes)
+    uint64_t p_full[2];   // 8 local warps + the peer's half of P (bytes)
     uint64_t p_free[2];   // PV done in both CTAs (multicast commit)
     uint64_t sx_full[2];  // the peer's partial scores (bytes)
     uint64_t sx_free[2];  // the peer consumed the partials this CTA sent
-    uint64_t lx_full, drain;
+    uint64_t lx_full, lx_loc, drain;
     uint32_t tmem_base;
     int abort;
     int max_slot;
@@ -86,10 +94,16 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(
 template <int NST, bool VSEP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnTcArgs a) {
+    static_assert(AT_SOFT0 % 4 == 0 && AT_PRODUCERS < AT_SOFT0, "warp roles");
     using Lay = AtLayout<NST, VSEP>;
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     AtBars* bars = (AtBars*)(smem + Lay::OFF_BAR);
+    uint32_t* vmask = (uint32_t*)(smem + Lay::OFF_VM);
+    if ((uintptr_t)smem != (uintptr_t)smem_raw) {  // the layout needs a 1024-byte aligned base
+        if (threadIdx.x == 0) report(a.st, DSA_ERR_UNSUPPORTED, -3);
+        return;
+    }
     const uint32_t warp = warp_id(), lane = lane_id();
     const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
     StatusHdr* st = a.st;
@@ -108,20 +122,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
-            mbar_init(smem_u32(&bars->full[i]), 64);
+            mbar_init(smem_u32(&bars->full[i]), AT_PRODUCERS * 32);
             mbar_init(smem_u32(&bars->empty[i]), 1);
         }
         mbar_init(smem_u32(&bars->s_full), 1);
-        mbar_init(smem_u32(&bars->s_empty), 4);
-        mbar_init(smem_u32(&bars->q_full), 4);
+        mbar_init(smem_u32(&bars->s_empty), 8);
+        mbar_init(smem_u32(&bars->q_full), 8);
         mbar_init(smem_u32(&bars->o_full), 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&bars->p_full[i]), 4);
+            mbar_init(smem_u32(&bars->p_full[i]), 8);
             mbar_init(smem_u32(&bars->p_free[i]), 2);
             mbar_init(smem_u32(&bars->sx_full[i]), 1);
-            mbar_init(smem_u32(&bars->sx_free[i]), 4);
+            mbar_init(smem_u32(&bars->sx_free[i]), 8);
         }
         mbar_init(smem_u32(&bars->lx_full), 1);
+        mbar_init(smem_u32(&bars->lx_loc), 8);
         mbar_init(smem_u32(&bars->drain), 1);
         // byte counts of the first phase of every peer-filled barrier
         for (int i = 0; i < 2; ++i) {
@@ -133,13 +148,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         bars->max_slot = -1;
         fence_mbar_init();
     }
-    if (warp == 2) tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) vmask[i] = 0u;
+    if (warp == AT_MMA_WARP) tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    // the softmax warps start their Q loads now; they land during the scan
+    uint4 qreg[8] = {};
+    const bool q_loader = warp >= AT_SOFT0;
+    const __nv_bfloat16* qrow = a.q + t * a.q_stride_tok + (int64_t)((warp & 3) * 32 + lane) * a.q_stride_head + col0;
+    if (q_loader) {  // block (warp - 3) >> 2 of this head's Q half
+        const uint4* src = (const uint4*)(qrow + 64 * (((int)warp - AT_SOFT0) >> 2));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qreg[i] = __ldg(src + i);
+    }
     __syncthreads();
-    // number of 64-slot tiles: up to the last valid slot of the index row
+    // validity bits of the index row and the number of 64-slot tiles (up to
+    // the last valid slot)
     {
         int m = -1;
-        for (int j = threadIdx.x; j < a.k_sel; j += blockDim.x)
-            if (__ldg(irow + j) >= 0) m = j;
+        for (int j0 = (int)(warp * 32); j0 < a.k_sel; j0 += (int)blockDim.x) {
+            const int j = j0 + (int)lane;
+            const int32_t v = j < a.k_sel ? __ldg(irow + j) : -1;
+            const uint32_t bits = __ballot_sync(0xffffffffu, v >= 0 && v < ri.seqlen_k);
+            if (v >= 0) m = j;
+            if (lane == 0 && j0 < 2048) vmask[j0 >> 5] = bits;
+        }
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0 && m >= 0) atomicMax(&bars->max_slot, m);
     }
@@ -151,36 +182,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 
     const uint32_t s_stage0 = smem_u32(smem);
     const uint32_t s_p0 = smem_u32(smem + Lay::OFF_P);
-    if (warp < 2) {
-        // ================= gather producers (64 threads) =================
-        const __nv_bfloat16* kbase = a.k;
-        const __nv_bfloat16* vbase = a.v;
-        const int key_in_warp = (int)(lane >> 3), chunk = (int)(lane & 7);
-        int32_t nxt = -1;
-        if (n_tiles > 0) {
-            const int slot = (int)(warp * 32 + lane);
-            nxt = slot < a.k_sel ? __ldg(irow + slot) : -1;
-        }
+    if (warp < AT_PRODUCERS) {
+        // ================= gather producers (7 warps) =================
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        // 16 groups of 4 keys per tile; warp w takes groups w, w+7, w+14
+        const int sub = (int)(lane >> 3), chunk = (int)(lane & 7);
+        const int ngrp = (16 - (int)warp + AT_PRODUCERS - 1) / AT_PRODUCERS;
+        int32_t nxt[3] = {-1, -1, -1};
+        auto load_idx = [&](int j) {
+#pragma unroll
+            for (int gi = 0; gi < 3; ++gi) {
+                const int slot = j * AT_N + 4 * ((int)warp + AT_PRODUCERS * gi) + sub;
+                nxt[gi] = (gi < ngrp && slot < a.k_sel) ? __ldg(irow + slot) : -1;
+            }
+        };
+        if (n_tiles > 0) load_idx(0);
         for (int j = 0; j < n_tiles; ++j) {
             const uint32_t s = j % NST;
-            int32_t v = nxt;
-            if (j + 1 < n_tiles) {
-                const int slot = (j + 1) * AT_N + (int)(warp * 32 + lane);
-                nxt = slot < a.k_sel ? __ldg(irow + slot) : -1;
-            }
-            if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
-            const int64_t row = ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0);
+            int32_t cur[3];
+#pragma unroll
+            for (int gi = 0; gi < 3; ++gi) cur[gi] = nxt[gi];
+            if (j + 1 < n_tiles) load_idx(j + 1);
             if (!wait_warp(smem_u32(&bars->empty[s]), ((j / NST) & 1) ^ 1, abort, st, 0x2101)) break;
             const uint32_t kst = s_stage0 + s * Lay::STAGE;
-#pragma unroll 1
-            for (int q = 0; q < 8; ++q) {
-                const int key = (int)(warp * 32) + 4 * q + key_in_warp;  // key of the tile
-                const int64_t r = __shfl_sync(0xffffffffu, row, 4 * q + key_in_warp);
-                const __nv_bfloat16* src = kbase + r * a.k_stride + col0 + chunk * 8;
+#pragma unroll
+            for (int gi = 0; gi < 3; ++gi) {
+                if (gi >= ngrp) break;
+                const int32_t v = cur[gi];
+                if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
+                const int64_t r = ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0);
+                const int key = 4 * ((int)warp + AT_PRODUCERS * gi) + sub;  // key of the tile
+                const __nv_bfloat16* src = a.k + r * a.k_stride + col0 + chunk * 8;
                 const uint32_t dst = kst + swz(key, chunk);
                 for (int kb = 0; kb < nb; ++kb) cp_async16(dst + kb * AT_BLK, src + kb * 64);
                 if (VSEP) {
-                    const __nv_bfloat16* vs = vbase + r * a.v_stride + dv0 + chunk * 8;
+                    const __nv_bfloat16* vs = a.v + r * a.v_stride + dv0 + chunk * 8;
 #pragma unroll
                     for (int vb = 0; vb < 4; ++vb) cp_async16(dst + AT_KST + vb * AT_BLK, vs + vb * 64);
                 }
@@ -188,8 +224,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             cp_async_arrive(smem_u32(&bars->full[s]));
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp == 2) {
+    } else if (warp == AT_MMA_WARP) {
         // ================= MMA issuer =================
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
         constexpr uint32_t idesc_s = idesc_make(1, 1, false, 128, AT_N);
         constexpr uint32_t idesc_pv = idesc_make(1, 1, true, 128, 256);
         // PV(t - kLag) follows S(t); S(t) reuses the stage PV(t - NST) frees,
@@ -199,7 +236,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         auto issue_pv = [&](int u) -> bool {
             const uint32_t b = u & 1;
             if (!wait_warp(smem_u32(&bars->p_full[b]), (u >> 1) & 1, abort, st, 0x2202)) return false;
-            fence_proxy_async();
             tc_fence_after();
             if (lane == 0) {
                 if (u + 2 < n_tiles) mbar_expect_tx(smem_u32(&bars->p_full[b]), AT_PX_BYTES);
@@ -241,37 +277,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             mbar_wait(smem_u32(&bars->drain), 0, nullptr, st, 0x2205, 1ll << 28);
         }
     } else {
-        // ================= softmax / exchange / epilogue =================
+        // ================= softmax / exchange / epilogue (8 warps) =================
+        // warps 8..11 and 12..15 each cover the four TMEM lane quadrants; the two
+        // warps of a quadrant split every tile's keys (hw = 0 / 1) and O's columns
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
         const uint32_t quad = warp & 3;
+        const int hw = (int)(warp - AT_SOFT0) >> 2;
         const int h = (int)(quad * 32 + lane);
         const uint32_t lane_off = (quad * 32) << 16;
         const int kh = (int)rank;  // this CTA's key half of every tile
         uint8_t* sx = smem + Lay::OFF_SX;
         const float* pmx = (const float*)(smem + Lay::OFF_PM);
-        const float* lx = (const float*)(smem + Lay::OFF_LX);
+        float* lx = (float*)(smem + Lay::OFF_LX);
         const uint32_t peer_sx = mapa(smem_u32(sx), peer);
         const uint32_t peer_pm = mapa(smem_u32(smem + Lay::OFF_PM), peer);
         const uint32_t peer_p = mapa(s_p0, peer);
-        const uint32_t peer_lx = mapa(smem_u32(smem + Lay::OFF_LX), peer);
         const uint32_t peer_sx_full0 = mapa(smem_u32(&bars->sx_full[0]), peer);
         const uint32_t peer_sx_free0 = mapa(smem_u32(&bars->sx_free[0]), peer);
         const uint32_t peer_p_full0 = mapa(smem_u32(&bars->p_full[0]), peer);
         const uint32_t peer_lx_full = mapa(smem_u32(&bars->lx_full), peer);
         const uint32_t my_sx_full0 = smem_u32(&bars->sx_full[0]), my_sx_free0 = smem_u32(&bars->sx_free[0]);
         const uint32_t my_p_full0 = smem_u32(&bars->p_full[0]), my_p_free0 = smem_u32(&bars->p_free[0]);
-        const bool arm_thread = threadIdx.x == 96;
+        const bool arm_thread = threadIdx.x == AT_SOFT0 * 32;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
-            // ---- Q half -> TMEM (A operand of S = Q K^T) ----
-            const __nv_bfloat16* qrow = a.q + t * a.q_stride_tok + (int64_t)h * a.q_stride_head + col0;
-            for (int kb = 0; kb < nb; ++kb) {
+            // ---- Q half -> TMEM (A operand of S = Q K^T); the quadrant's two warps
+            // take alternate 64-column blocks, block hw was loaded early ----
+            for (int kb = hw; kb < nb; kb += 2) {
                 uint32_t r[32];
-                const uint4* src = (const uint4*)(qrow + kb * 64);
+                if (kb > 1) {
+                    const uint4* src = (const uint4*)(qrow + kb * 64);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) qreg[i] = __ldg(src + i);
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint4 v = __ldg(src + i);
-                    r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+                    r[4 * i] = qreg[i].x; r[4 * i + 1] = qreg[i].y; r[4 * i + 2] = qreg[i].z; r[4 * i + 3] = qreg[i].w;
                 }
                 tmem_st32(tmem + lane_off + TM_Q + kb * 32, r);
             }
@@ -280,25 +322,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
         }
-        // per-tile data carried from stage A to stage B
-        float mine_cur[32], mine_nxt[32];
+        // per-tile data carried from stage A to stage B: this warp's 16 keys
+        float mine_cur[16], mine_nxt[16];
         float pm_cur = -INFINITY, pm_nxt = -INFINITY;
         uint32_t msk_cur = 0, msk_nxt = 0;
-        int32_t iv0 = -1, iv1 = -1;  // slots of the next tile to read
-        if (n_tiles > 0) {
-            iv0 = (int)lane < a.k_sel ? __ldg(irow + lane) : -1;
-            iv1 = (int)lane + 32 < a.k_sel ? __ldg(irow + lane + 32) : -1;
-        }
-        // Stage A of tile u: read S, partial max, send the peer's half.
+        // Stage A of tile u: read S, full-row partial max, send the peer's keys of this warp.
         auto stage_a = [&](int u) -> bool {
             const uint32_t b = u & 1, ph = (u >> 1) & 1;
-            const uint32_t mlo = __ballot_sync(0xffffffffu, iv0 >= 0 && iv0 < ri.seqlen_k);
-            const uint32_t mhi = __ballot_sync(0xffffffffu, iv1 >= 0 && iv1 < ri.seqlen_k);
-            if (u + 1 < n_tiles) {  // prefetch the following tile's slots
-                const int sl0 = (u + 1) * AT_N + (int)lane, sl1 = sl0 + 32;
-                iv0 = sl0 < a.k_sel ? __ldg(irow + sl0) : -1;
-                iv1 = sl1 < a.k_sel ? __ldg(irow + sl1) : -1;
-            }
+            const uint32_t mlo = u < 32 ? vmask[2 * u] : 0u, mhi = u < 32 ? vmask[2 * u + 1] : 0u;
             if (!wait_warp(smem_u32(&bars->s_full), u & 1, abort, st, 0x2301)) return false;
             tc_fence_after();
             uint32_t r0[32], r1[32];
@@ -317,41 +348,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             if (!wait_warp(my_sx_free0 + 8 * b, ph ^ 1, abort, st, 0x2302)) return false;
             const uint32_t dst = peer_sx + b * AT_TILE128;
             const uint32_t bar = peer_sx_full0 + 8 * b;
+            // the peer's keys are [32,64) for rank 0, [0,32) for rank 1; this warp sends 16 of them
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {  // the peer's keys: [32,64) for rank 0, [0,32) for rank 1
+            for (int c = 0; c < 4; ++c) {
                 uint32_t w[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
-                st_async_v4(dst + swz(h, c), w[0], w[1], w[2], w[3], bar);
+                for (int e = 0; e < 4; ++e)
+                    w[e] = kh ? (hw ? r0[16 + 4 * c + e] : r0[4 * c + e]) : (hw ? r1[16 + 4 * c + e] : r1[4 * c + e]);
+                st_async_v4(dst + swz(h, 4 * hw + c), w[0], w[1], w[2], w[3], bar);
             }
-            st_async_b32(peer_pm + b * 512 + h * 4, __float_as_uint(pm), bar);
+            if (hw == 0) st_async_b32(peer_pm + b * 512 + h * 4, __float_as_uint(pm), bar);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mine_nxt[i] = __uint_as_float(kh ? r1[i] : r0[i]);
+            for (int i = 0; i < 16; ++i)
+                mine_nxt[i] = __uint_as_float(kh ? (hw ? r1[16 + i] : r1[i]) : (hw ? r0[16 + i] : r0[i]));
             pm_nxt = pm;
-            msk_nxt = kh ? mhi : mlo;
+            msk_nxt = ((kh ? mhi : mlo) >> (16 * hw)) & 0xFFFFu;
             return true;
         };
-        // Stage B of tile u: combine, probabilities, write both copies of P.
+        // Stage B of tile u: combine, probabilities, write both copies of this warp's P part.
         auto stage_b = [&](int u) -> bool {
             const uint32_t b = u & 1, ph = (u >> 1) & 1;
             if (!wait_warp(my_sx_full0 + 8 * b, ph, abort, st, 0x2303)) return false;
             if (arm_thread && u + 2 < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * b, AT_SX_BYTES);
-            float s32[32];
+            float s16[16];
             {
                 const uint8_t* rowp = sx + b * AT_TILE128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 v = *(const float4*)(rowp + swz(h, c));
-                    s32[4 * c] = mine_cur[4 * c] + v.x;
-                    s32[4 * c + 1] = mine_cur[4 * c + 1] + v.y;
-                    s32[4 * c + 2] = mine_cur[4 * c + 2] + v.z;
-                    s32[4 * c + 3] = mine_cur[4 * c + 3] + v.w;
+                for (int c = 0; c < 4; ++c) {
+                    const float4 v = *(const float4*)(rowp + swz(h, 4 * hw + c));
+                    s16[4 * c] = mine_cur[4 * c] + v.x;
+                    s16[4 * c + 1] = mine_cur[4 * c + 1] + v.y;
+                    s16[4 * c + 2] = mine_cur[4 * c + 2] + v.z;
+                    s16[4 * c + 3] = mine_cur[4 * c + 3] + v.w;
                 }
             }
             const float pm_peer = pmx[b * 128 + h];
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * b);
-            // shared running maximum (identical in both CTAs), lazy rescale
+            // shared running maximum (identical in all four warps of a head), lazy rescale
             const float mb = (pm_cur == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm_cur + pm_peer) * a.scale_log2;
             float alpha = 1.f;
             if (mb > m_used + 8.0f) {
@@ -359,13 +393,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 l *= alpha;
                 m_used = mb;
             }
-            uint32_t pw[16];
+            uint32_t pw[8];
             {
                 float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = ((msk_cur >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
-                    const float p1 = ((msk_cur >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
+                for (int i = 0; i < 8; ++i) {
+                    const float p0 = ((msk_cur >> (2 * i)) & 1u) ? ex2(fmaf(s16[2 * i], a.scale_log2, -m_used)) : 0.f;
+                    const float p1 = ((msk_cur >> (2 * i + 1)) & 1u) ? ex2(fmaf(s16[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
                     rs0 += p0;
                     rs1 += p1;
                     pw[i] = pack_bf16(p0, p1);
@@ -379,24 +413,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 const uint32_t pdst = peer_p + b * AT_TILE128;
                 const uint32_t bar = peer_p_full0 + 8 * b;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = 4 * kh + q;
+                for (int q = 0; q < 2; ++q) {
+                    const int c = 4 * kh + 2 * hw + q;
                     *(uint4*)(prow + swz(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
                     st_async_v4(pdst + swz(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
                 }
             }
             if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                // O may be rescaled only between PV(u-1) and PV(u)
+                // O may be rescaled only between PV(u-1) and PV(u); this warp owns 128 columns
                 const int w = u - 1;
                 if (!wait_warp(my_p_free0 + 8 * (w & 1), (w >> 1) & 1, abort, st, 0x2305)) return false;
                 tc_fence_after();
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + TM_O + c * 32, r);
+                    const uint32_t ta = tmem + lane_off + TM_O + 128 * hw + c * 32;
+                    tmem_ld32(ta, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(tmem + lane_off + TM_O + c * 32, r);
+                    tmem_st32(ta, r);
                 }
                 tmem_wait_st();
             }
@@ -409,28 +444,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         if (n_tiles > 0) ok = stage_a(0);
         for (int j = 0; ok && j < n_tiles; ++j) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mine_cur[i] = mine_nxt[i];
+            for (int i = 0; i < 16; ++i) mine_cur[i] = mine_nxt[i];
             pm_cur = pm_nxt;
             msk_cur = msk_nxt;
             if (j + 1 < n_tiles && !stage_a(j + 1)) { ok = false; break; }
             if (!stage_b(j)) { ok = false; break; }
         }
-        // ---- row sums of both halves ----
+        // ---- row sums: this CTA's two partials, then the peer's sum ----
         float l_tot = 0.f;
         if (ok && n_tiles > 0) {
-            st_async_b32(peer_lx + h * 4, __float_as_uint(l), peer_lx_full);
-            if (wait_warp(smem_u32(&bars->lx_full), 0, abort, st, 0x2306)) l_tot = l + lx[h];
+            lx[hw * 128 + h] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->lx_loc));
+            ok = wait_warp(smem_u32(&bars->lx_loc), 0, abort, st, 0x2306);
+            const float l_cta = lx[h] + lx[128 + h];
+            // the peer's sum lands in partial-max buffer n_tiles & 1, free once the
+            // peer has consumed this CTA's partials of tile n_tiles - 2
+            const uint32_t bf = n_tiles & 1;
+            if (ok && hw == 0) {
+                ok = wait_warp(my_sx_free0 + 8 * bf, ((n_tiles >> 1) & 1) ^ 1, abort, st, 0x2307);
+                if (ok) st_async_b32(peer_pm + bf * 512 + h * 4, __float_as_uint(l_cta), peer_lx_full);
+            }
+            if (ok && wait_warp(smem_u32(&bars->lx_full), 0, abort, st, 0x2308)) l_tot = l_cta + pmx[bf * 128 + h];
             else ok = false;
         }
-        // ---- epilogue: O / l -> bf16 ----
-        __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0;
+        // ---- epilogue: O / l -> bf16 (this warp's 128 output columns) ----
+        __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + 128 * hw;
         const bool have_o = ok && n_tiles > 0 && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2307);
         if (have_o) tc_fence_after();
         const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
             if (have_o) {
-                tmem_ld32(tmem + lane_off + TM_O + c * 32, r);
+                tmem_ld32(tmem + lane_off + TM_O + 128 * hw + c * 32, r);
                 tmem_wait_ld();
             }
             uint4* dst = (uint4*)(orow + c * 32);
@@ -448,14 +494,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 dst[i] = w;
             }
         }
-        if (rank == 0 && a.lse)
+        if (rank == 0 && hw == 0 && a.lse)
             a.lse[t * 128 + h] = (have_o && l_tot > 0.f) ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
     }
     tc_fence_before();
     __syncwarp();
     cluster_sync();  // no DSMEM traffic may target a CTA that has exited
     tc_fence_after();
-    if (warp == 2) tmem_dealloc(tmem, 512);
+    if (warp == AT_MMA_WARP) tmem_dealloc(tmem, 512);
 }
 
 template <int NST, bool VSEP>
