@@ -185,6 +185,31 @@ DSA_API int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const
 DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
                        int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* dsa_select without a workspace, for callers that cannot allocate device
+ * memory: code running inside a host framework that owns every byte of the
+ * GPU through its own pool and allows no further cudaMalloc (an inference
+ * engine's plugin, for example), or a latency-critical path that must not
+ * pay for an allocation.  This entry point has no counterpart in the paper;
+ * it is a deployment convenience of this library.
+ *
+ * Same result as dsa_select.  Only prefill-shaped E4M3 inputs
+ * (max_seqlen_q >= 64, the fused tensor-core indexer) are served, with at
+ * most 32768 query rows in total; more rows return DSA_ERR_WORKSPACE, other
+ * shapes DSA_ERR_UNSUPPORTED, and nothing is launched.
+ *
+ * The scratch it needs (a status header, the folded query codes and their
+ * scales: about 4.3 MB) is a static array inside the library that every GPU
+ * loading the library keeps until the process exits.  The first call on a
+ * device looks up that array's device address (once per device); make that
+ * first call before any stream capture begins.  All calls share the one
+ * array, so calls whose work overlaps on the GPU (other streams, other host
+ * threads) race; serialise them.  The status header is cleared at the start
+ * of every call.  The call allocates nothing, waits for `stream` to finish
+ * the work, and returns the device-side status (DSA_OK, DSA_ERR_TIMEOUT,
+ * DSA_ERR_INDEX) or a validation / CUDA error. */
+DSA_API int dsa_select_noalloc(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
+                               int64_t ld_idx, dsa_stream_t stream);
+
 /* The whole hot path: a1 fold -> a2+a3 fused indexer/top-k (the scores stay
  * on chip) -> a4 sparse attention.  idx_out (nullable; int32
  * [total_q, ld_idx]) receives the selected indices as dsa_topk would

@@ -443,3 +443,66 @@ int dsa_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t budget_cycles, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// dsa_select_noalloc: dsa_select for callers that cannot allocate device
+// memory.  Its scratch (status header, folded query codes and their scales)
+// is the static device array below; see include/dsa.h for the contract.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+constexpr int64_t kNoAllocMaxRows = 32768;
+constexpr size_t kNoAllocU = kHdr;                                        // e4m3 [rows,128]
+constexpr size_t kNoAllocS = kNoAllocU + (size_t)kNoAllocMaxRows * 128;  // fp32 [rows]
+constexpr size_t kNoAllocBytes = kNoAllocS + (size_t)kNoAllocMaxRows * 4;
+constexpr int kNoAllocMaxDevices = 64;
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices];  // device address of the array, per device
+
+// Device address of the scratch array on the current device, looked up once
+// per device with that device current (a host-side reference to the array
+// is only a stand-in and must never be passed to a kernel).
+int noalloc_scratch(uint8_t** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return DSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = (uint8_t*)g_noalloc_ptr[dev];
+    return DSA_OK;
+}
+}  // namespace
+
+extern "C" int dsa_select_noalloc(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
+                                  int64_t ld_idx, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_indexer(seqs, ia);
+    if (r) return r;
+    if (k < 1 || (seqs->total_q && (!idx || ld_idx < k))) return DSA_ERR_INVALID_ARG;
+    if (!use_tc_indexer(seqs, ia)) return DSA_ERR_UNSUPPORTED;  // needs the fused (no score buffer) path
+    if (seqs->total_q > kNoAllocMaxRows) return DSA_ERR_WORKSPACE;
+    if (seqs->total_q == 0) return DSA_OK;
+    uint8_t* w = nullptr;
+    r = noalloc_scratch(&w);
+    if (r) return r;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the status header must start at zero; the code rows are rewritten in full
+    if (cudaMemsetAsync(w, 0, kHdr, st) != cudaSuccess) return DSA_ERR_CUDA;
+    r = run_fold(seqs, ia, w + kNoAllocU, (float*)(w + kNoAllocS), st);
+    if (!r)
+        r = run_indexer_tc(seqs, ia, w + kNoAllocU, (const float*)(w + kNoAllocS), 0, k, idx, ld_idx, nullptr, 0, 0, 0,
+                           hdr(w), st);
+    if (r) return r;
+    StatusHdr h;
+    if (cudaMemcpyAsync(&h, w, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    return h.code;
+}

@@ -51,15 +51,17 @@ _lib.dsa_topk.argtypes = [_S, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_sparse_attn.argtypes = [_S, _AA, _P, _I64, _I32, _P, _SZ, _P]
 _lib.dsa_forward.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_select.argtypes = [_S, _IA, _I32, _P, _I64, _P, _SZ, _P]
+_lib.dsa_select_noalloc.argtypes = [_S, _IA, _I32, _P, _I64, _P]
 _lib.dsa_sync_status.argtypes = [_P, _P, ctypes.POINTER(_I64)]
 _lib.dsa_selftest_wait_timeout.argtypes = [_P, _SZ, _I64, _P]
 for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
-           "dsa_select",
+           "dsa_select", "dsa_select_noalloc",
            "dsa_sync_status", "dsa_selftest_wait_timeout"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk",
-            "dsa_sparse_attn", "dsa_forward", "dsa_select", "dsa_sync_status", "dsa_selftest_wait_timeout")
+            "dsa_sparse_attn", "dsa_forward", "dsa_select", "dsa_select_noalloc", "dsa_sync_status",
+            "dsa_selftest_wait_timeout")
 
 
 class DsaError(RuntimeError):
@@ -182,6 +184,13 @@ def dsa_forward(seqs, ia, aa, k, idx_out, ws):
 def dsa_select(seqs, ia, k, idx, ws):
     _check(_lib.dsa_select(ctypes.byref(seqs.c), ctypes.byref(ia), k, _ptr(idx), idx.stride(0), _ptr(ws), ws.numel(),
                            _stream()), "dsa_select")
+
+
+def dsa_select_noalloc(seqs, ia, k, idx):
+    """dsa_select without a workspace (for callers that cannot allocate device
+    memory): synchronous, returns nothing, raises DsaError on any status."""
+    _check(_lib.dsa_select_noalloc(ctypes.byref(seqs.c), ctypes.byref(ia), k, _ptr(idx), idx.stride(0), _stream()),
+           "dsa_select_noalloc")
 
 
 def dsa_sync_status(ws):
