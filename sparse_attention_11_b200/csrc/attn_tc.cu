@@ -26,10 +26,10 @@
 // hold the full 128 x 64 P (the A operand of O += P V, in shared memory).
 // Row sums are combined once at the end.
 //
-// Pipelining.  The softmax warps run stage A of tile j+1 (read S, send the
-// partial) before stage B of tile j (combine, probabilities, write P), so each
-// exchange has a whole stage to land; the MMA warp issues S(t) then PV(t-2)
-// (PV(t-1) with only two K/V stages).
+// Pipelining.  Stage A (read S, send the partial) and stage B (combine,
+// probabilities, write P) run in separate warps, so consecutive tiles overlap;
+// the MMA warp issues greedily: PV(u) as soon as P(u) is complete, else S(t)
+// as soon as its K/V stage is full and the S buffer is free.
 // P tiles are double-buffered and released by a tcgen05.commit that arrives
 // on the p_free barrier of both CTAs (PV(t) done in both), so stage B waits
 // for PV(t-2), and for PV(t-1) only when the running maximum moves.
@@ -41,10 +41,11 @@
 // warps, so the producers are many and small (setmaxnreg moves their
 // registers to the softmax warps).
 //
-// Tensor memory per CTA: O [0,256)  S [256,320)  Q [320, 320 + 32 * blocks).
+// Tensor memory per CTA: O [0,256)  S [256,384) (two buffers)  Q [384,512)
+// (four 64-column blocks; rank 1's fifth block, the rope part, is read from
+// shared memory by SS MMAs).
 // Warps: 0-6 producers, 7 MMA issuer (+TMEM owner), 8-15 softmax / exchange /
-// epilogue: two warps per TMEM lane quadrant (thread <-> head), splitting
-// each tile's keys and O's columns.
+// epilogue: an A and a B warp per TMEM lane quadrant (thread <-> head).
 #include "dsa_kernels.h"
 
 namespace dsa {
@@ -56,19 +57,20 @@ constexpr uint32_t AT_VST = 4 * AT_BLK;            // V part (separate V only)
 constexpr uint32_t AT_TILE128 = 128 * 128;         // a 128-row x 128-byte swizzled tile
 constexpr uint32_t AT_SX_BYTES = 128 * 128 + 128 * 4;  // partial scores + partial maxima
 constexpr uint32_t AT_PX_BYTES = 128 * 64;         // the peer's half of P
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320;
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;  // S: two 64-column buffers
 constexpr int AT_THREADS = 512;  // 7 producer + 1 MMA + 8 softmax warps
 constexpr int AT_PRODUCERS = 7;
 constexpr int AT_MMA_WARP = 7;
 constexpr int AT_SOFT0 = 8;     // first softmax warp (a warpgroup boundary)
 
-template <int NST, bool VSEP>
+template <int NST, bool VSEP, int NPB = 2, int NSX = 2>
 struct AtLayout {
     static constexpr uint32_t STAGE = AT_KST + (VSEP ? AT_VST : 0);
-    static constexpr uint32_t OFF_P = NST * STAGE;            // [2] P tiles
-    static constexpr uint32_t OFF_SX = OFF_P + 2 * AT_TILE128;  // [2] partial-score tiles
-    static constexpr uint32_t OFF_PM = OFF_SX + 2 * AT_TILE128; // [2][128] partial maxima
-    static constexpr uint32_t OFF_LX = OFF_PM + 2 * 512;        // [2][128] this CTA's row-sum partials
+    static constexpr uint32_t OFF_QR = NST * STAGE;           // rank 1's 5th Q block (rope), A of SS MMAs
+    static constexpr uint32_t OFF_P = OFF_QR + AT_TILE128;    // [NPB] P tiles
+    static constexpr uint32_t OFF_SX = OFF_P + NPB * AT_TILE128;  // [NSX] partial-score tiles
+    static constexpr uint32_t OFF_PM = OFF_SX + NSX * AT_TILE128; // [NSX][128] partial maxima
+    static constexpr uint32_t OFF_LX = OFF_PM + NSX * 512;        // [128] row sums for the A warps' epilogue
     static constexpr uint32_t OFF_VM = OFF_LX + 1024;            // [64] validity bits of 2048 slots
     static constexpr uint32_t OFF_BAR = OFF_VM + 256;
     static constexpr uint32_t SMEM = OFF_BAR + 256;
@@ -77,8 +79,8 @@ struct AtLayout {
 struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
-    uint64_t s_full, s_empty, q_full, o_full;
-    uint64_t p_full[2];   // 8 local warps + the peer's half of P (bytes)
+    uint64_t s_full[2], s_empty[2], q_full, o_full;
+    uint64_t p_full[2];   // 4 local B warps + the peer's half of P (bytes)
     uint64_t p_free[2];   // PV done in both CTAs (multicast commit)
     uint64_t sx_full[2];  // the peer's partial scores (bytes)
     uint64_t sx_free[2];  // the peer consumed the partials this CTA sent
@@ -91,11 +93,11 @@ static_assert(sizeof(AtBars) <= 256, "barrier block");
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 
-template <int NST, bool VSEP>
+template <int NST, bool VSEP, int NPB, int NSX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnTcArgs a) {
     static_assert(AT_SOFT0 % 4 == 0 && AT_PRODUCERS < AT_SOFT0, "warp roles");
-    using Lay = AtLayout<NST, VSEP>;
+    using Lay = AtLayout<NST, VSEP, NPB, NSX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     AtBars* bars = (AtBars*)(smem + Lay::OFF_BAR);
@@ -125,22 +127,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             mbar_init(smem_u32(&bars->full[i]), AT_PRODUCERS * 32);
             mbar_init(smem_u32(&bars->empty[i]), 1);
         }
-        mbar_init(smem_u32(&bars->s_full), 1);
-        mbar_init(smem_u32(&bars->s_empty), 8);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bars->s_full[i]), 1);
+            mbar_init(smem_u32(&bars->s_empty[i]), 8);  // 4 A + 4 B warps read every S tile
+        }
         mbar_init(smem_u32(&bars->q_full), 8);
         mbar_init(smem_u32(&bars->o_full), 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&bars->p_full[i]), 8);
+            mbar_init(smem_u32(&bars->p_full[i]), 4);  // (only NPB of them are used)
             mbar_init(smem_u32(&bars->p_free[i]), 2);
             mbar_init(smem_u32(&bars->sx_full[i]), 1);
-            mbar_init(smem_u32(&bars->sx_free[i]), 8);
+            mbar_init(smem_u32(&bars->sx_free[i]), 4);
         }
         mbar_init(smem_u32(&bars->lx_full), 1);
-        mbar_init(smem_u32(&bars->lx_loc), 8);
+        mbar_init(smem_u32(&bars->lx_loc), 4);
         mbar_init(smem_u32(&bars->drain), 1);
         // byte counts of the first phase of every peer-filled barrier
-        for (int i = 0; i < 2; ++i) {
-            mbar_expect_tx(smem_u32(&bars->p_full[i]), AT_PX_BYTES);
+        for (int i = 0; i < NPB; ++i) mbar_expect_tx(smem_u32(&bars->p_full[i]), AT_PX_BYTES);
+        for (int i = 0; i < NSX; ++i) {
             mbar_arrive_expect_tx(smem_u32(&bars->sx_full[i]), AT_SX_BYTES);
         }
         mbar_arrive_expect_tx(smem_u32(&bars->lx_full), 128 * 4);
@@ -182,6 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 
     const uint32_t s_stage0 = smem_u32(smem);
     const uint32_t s_p0 = smem_u32(smem + Lay::OFF_P);
+    const uint32_t s_qr = smem_u32(smem + Lay::OFF_QR);
     if (warp < AT_PRODUCERS) {
         // ================= gather producers (7 warps) =================
         asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
@@ -229,48 +234,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
         constexpr uint32_t idesc_s = idesc_make(1, 1, false, 128, AT_N);
         constexpr uint32_t idesc_pv = idesc_make(1, 1, true, 128, 256);
-        // PV(t - kLag) follows S(t); S(t) reuses the stage PV(t - NST) frees,
-        // so the lag must stay below the stage count.
-        constexpr int kLag = NST >= 3 ? 2 : 1;
         bool ok = n_tiles > 0 && wait_warp(smem_u32(&bars->q_full), 0, abort, st, 0x2201);
-        auto issue_pv = [&](int u) -> bool {
-            const uint32_t b = u & 1;
-            if (!wait_warp(smem_u32(&bars->p_full[b]), (u >> 1) & 1, abort, st, 0x2202)) return false;
-            tc_fence_after();
-            if (lane == 0) {
-                if (u + 2 < n_tiles) mbar_expect_tx(smem_u32(&bars->p_full[b]), AT_PX_BYTES);
-                const uint32_t vb = s_stage0 + (u % NST) * Lay::STAGE + (VSEP ? AT_KST : 0);
-                const uint32_t pb = s_p0 + b * AT_TILE128;
+        // Greedy issue: PV(ju) as soon as its P tile is complete (ju < js), else
+        // S(js) as soon as its K/V stage is full and the S buffer is free.
+        int js = 0, ju = 0;
+        long long idle0 = clock64();
+        while (ok && ju < n_tiles) {
+            bool done = false;
+            if (ju < js) {
+                const uint32_t b = ju % NPB;
+                if (__all_sync(0xffffffffu, mbar_probe(smem_u32(&bars->p_full[b]), (ju / NPB) & 1))) {
+                    tc_fence_after();
+                    if (lane == 0) {
+                        if (ju + NPB < n_tiles) mbar_expect_tx(smem_u32(&bars->p_full[b]), AT_PX_BYTES);
+                        const uint32_t vb = s_stage0 + (ju % NST) * Lay::STAGE + (VSEP ? AT_KST : 0);
+                        const uint32_t pb = s_p0 + b * AT_TILE128;
 #pragma unroll
-                for (int ks = 0; ks < AT_N / 16; ++ks)
-                    mma_bf16_ss(tmem + TM_O, sdesc_sw128(pb + ks * 32, 16, 1024), sdesc_sw128(vb + ks * 2048, AT_BLK, 1024),
-                                idesc_pv, (u > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(smem_u32(&bars->empty[u % NST]));
-                mma_commit_mc(smem_u32(&bars->p_free[b]), (uint16_t)3);
+                        for (int ks = 0; ks < AT_N / 16; ++ks)
+                            mma_bf16_ss(tmem + TM_O, sdesc_sw128(pb + ks * 32, 16, 1024),
+                                        sdesc_sw128(vb + ks * 2048, AT_BLK, 1024), idesc_pv, (ju > 0 || ks > 0) ? 1u : 0u);
+                        mma_commit(smem_u32(&bars->empty[ju % NST]));
+                        mma_commit_mc(smem_u32(&bars->p_free[b]), (uint16_t)3);
+                    }
+                    __syncwarp();
+                    ++ju;
+                    done = true;
+                }
             }
-            __syncwarp();
-            return true;
-        };
-        for (int j = 0; ok && j < n_tiles; ++j) {
-            const uint32_t s = j % NST;
-            if (!wait_warp(smem_u32(&bars->full[s]), (j / NST) & 1, abort, st, 0x2203)) { ok = false; break; }
-            fence_proxy_async();
-            if (!wait_warp(smem_u32(&bars->s_empty), (j & 1) ^ 1, abort, st, 0x2204)) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t kst = s_stage0 + s * Lay::STAGE;
-                for (int kb = 0; kb < nb; ++kb)
+            if (!done && js < n_tiles) {
+                const uint32_t s = js % NST, sb = js & 1;
+                const bool rdy = mbar_probe(smem_u32(&bars->full[s]), (js / NST) & 1) &&
+                                 mbar_probe(smem_u32(&bars->s_empty[sb]), ((js >> 1) & 1) ^ 1);
+                if (__all_sync(0xffffffffu, rdy)) {
+                    fence_proxy_async();
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t kst = s_stage0 + s * Lay::STAGE;
+                        const uint32_t d = tmem + TM_S + 64 * sb;
+                        for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16_ts(tmem + TM_S, tmem + TM_Q + kb * 32 + ks * 8,
-                                    sdesc_sw128(kst + kb * AT_BLK + ks * 32, 16, 1024), idesc_s, (kb | ks) ? 1u : 0u);
-                mma_commit(smem_u32(&bars->s_full));
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16_ts(d, tmem + TM_Q + kb * 32 + ks * 8, sdesc_sw128(kst + kb * AT_BLK + ks * 32, 16, 1024),
+                                            idesc_s, (kb | ks) ? 1u : 0u);
+                        if (nb == 5)  // the rope block: Q from shared memory
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16_ss(d, sdesc_sw128(s_qr + ks * 32, 16, 1024),
+                                            sdesc_sw128(kst + 4 * AT_BLK + ks * 32, 16, 1024), idesc_s, 1u);
+                        mma_commit(smem_u32(&bars->s_full[sb]));
+                    }
+                    __syncwarp();
+                    ++js;
+                    done = true;
+                }
             }
-            __syncwarp();
-            if (j >= kLag && !issue_pv(j - kLag)) { ok = false; break; }
+            if (done) {
+                idle0 = clock64();
+            } else {
+                const long long el = clock64() - idle0;
+                bool give_up = *abort != 0;
+                if (!give_up && el > (1ll << 20) && *(volatile int*)&st->code == DSA_ERR_TIMEOUT) give_up = true;
+                if (!give_up && el > kWaitBudget) {
+                    report(st, DSA_ERR_TIMEOUT, 0x2203);
+                    give_up = true;
+                }
+                if (__any_sync(0xffffffffu, give_up)) {
+                    *abort = 1;
+                    ok = false;
+                }
+            }
         }
-        for (int u = n_tiles >= kLag ? n_tiles - kLag : 0; ok && u < n_tiles; ++u)
-            if (!issue_pv(u)) ok = false;
         if (ok && n_tiles > 0 && lane == 0) mma_commit(smem_u32(&bars->o_full));
         if (*abort && lane == 0) {
             mma_commit(smem_u32(&bars->drain));
@@ -278,11 +311,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         }
     } else {
         // ================= softmax / exchange / epilogue (8 warps) =================
-        // warps 8..11 and 12..15 each cover the four TMEM lane quadrants; the two
-        // warps of a quadrant split every tile's keys (hw = 0 / 1) and O's columns
+        // Stage-specialised: warps 8..11 ("A", one per TMEM lane quadrant) read
+        // each S tile, form the row's partial maximum and send the peer's 32
+        // partial columns; warps 12..15 ("B") read their own 32 columns of the
+        // same tile, combine them with the peer's partials, form the
+        // probabilities and write P.  Both groups run every tile concurrently.
         asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
         const uint32_t quad = warp & 3;
-        const int hw = (int)(warp - AT_SOFT0) >> 2;
+        const bool is_b = warp >= AT_SOFT0 + 4;
         const int h = (int)(quad * 32 + lane);
         const uint32_t lane_off = (quad * 32) << 16;
         const int kh = (int)rank;  // this CTA's key half of every tile
@@ -298,13 +334,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         const uint32_t peer_lx_full = mapa(smem_u32(&bars->lx_full), peer);
         const uint32_t my_sx_full0 = smem_u32(&bars->sx_full[0]), my_sx_free0 = smem_u32(&bars->sx_free[0]);
         const uint32_t my_p_full0 = smem_u32(&bars->p_full[0]), my_p_free0 = smem_u32(&bars->p_free[0]);
-        const bool arm_thread = threadIdx.x == AT_SOFT0 * 32;
+        const bool arm_thread = threadIdx.x == (AT_SOFT0 + 4) * 32;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
-            // ---- Q half -> TMEM (A operand of S = Q K^T); the quadrant's two warps
-            // take alternate 64-column blocks, block hw was loaded early ----
-            for (int kb = hw; kb < nb; kb += 2) {
+            // ---- Q half -> TMEM (A operand of S = Q K^T); the A and B warps of a
+            // quadrant take alternate 64-column blocks, block (is_b) was loaded early ----
+            for (int kb = is_b ? 1 : 0; kb < nb; kb += 2) {
                 uint32_t r[32];
                 if (kb > 1) {
                     const uint4* src = (const uint4*)(qrow + kb * 64);
@@ -315,118 +351,117 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 for (int i = 0; i < 8; ++i) {
                     r[4 * i] = qreg[i].x; r[4 * i + 1] = qreg[i].y; r[4 * i + 2] = qreg[i].z; r[4 * i + 3] = qreg[i].w;
                 }
-                tmem_st32(tmem + lane_off + TM_Q + kb * 32, r);
+                if (kb < 4) {
+                    tmem_st32(tmem + lane_off + TM_Q + kb * 32, r);
+                } else {
+                    uint8_t* qr = smem + Lay::OFF_QR;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *(uint4*)(qr + swz(h, c)) = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+                }
             }
             tmem_wait_st();
+            fence_proxy_async();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
         }
-        // per-tile data carried from stage A to stage B: this warp's 16 keys
-        float mine_cur[16], mine_nxt[16];
-        float pm_cur = -INFINITY, pm_nxt = -INFINITY;
-        uint32_t msk_cur = 0, msk_nxt = 0;
-        // Stage A of tile u: read S, full-row partial max, send the peer's keys of this warp.
-        auto stage_a = [&](int u) -> bool {
-            const uint32_t b = u & 1, ph = (u >> 1) & 1;
+        for (int u = 0; ok && u < n_tiles; ++u) {
+            const uint32_t b = u & 1, ph = (u >> 1) & 1;  // S buffer and its phase
+            const uint32_t xb = u % NSX, xph = (u / NSX) & 1;  // partial-score buffer and its phase
             const uint32_t mlo = u < 32 ? vmask[2 * u] : 0u, mhi = u < 32 ? vmask[2 * u + 1] : 0u;
-            if (!wait_warp(smem_u32(&bars->s_full), u & 1, abort, st, 0x2301)) return false;
+            if (!wait_warp(smem_u32(&bars->s_full[b]), ph, abort, st, 0x2301)) { ok = false; break; }
             tc_fence_after();
             uint32_t r0[32], r1[32];
-            tmem_ld32(tmem + lane_off + TM_S, r0);
-            tmem_ld32(tmem + lane_off + TM_S + 32, r1);
+            tmem_ld32(tmem + lane_off + TM_S + 64 * b, r0);
+            tmem_ld32(tmem + lane_off + TM_S + 64 * b + 32, r1);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
-            float pm = -INFINITY;
+            if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b]));
+            float pm = -INFINITY;  // partial maximum of this CTA's row over the tile's valid keys
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 if ((mlo >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r0[i]));
                 if ((mhi >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r1[i]));
             }
-            if (!wait_warp(my_sx_free0 + 8 * b, ph ^ 1, abort, st, 0x2302)) return false;
-            const uint32_t dst = peer_sx + b * AT_TILE128;
-            const uint32_t bar = peer_sx_full0 + 8 * b;
-            // the peer's keys are [32,64) for rank 0, [0,32) for rank 1; this warp sends 16 of them
+            if (!is_b) {
+                // ---- stage A: send the peer's 32 partial columns and the partial max ----
+                if (!wait_warp(my_sx_free0 + 8 * xb, xph ^ 1, abort, st, 0x2302)) { ok = false; break; }
+                const uint32_t dst = peer_sx + xb * AT_TILE128;
+                const uint32_t bar = peer_sx_full0 + 8 * xb;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t w[4];
+                for (int c = 0; c < 8; ++c) {  // the peer's keys: [32,64) for rank 0, [0,32) for rank 1
+                    uint32_t w[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w[e] = kh ? (hw ? r0[16 + 4 * c + e] : r0[4 * c + e]) : (hw ? r1[16 + 4 * c + e] : r1[4 * c + e]);
-                st_async_v4(dst + swz(h, 4 * hw + c), w[0], w[1], w[2], w[3], bar);
+                    for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
+                    st_async_v4(dst + swz(h, c), w[0], w[1], w[2], w[3], bar);
+                }
+                st_async_b32(peer_pm + xb * 512 + h * 4, __float_as_uint(pm), bar);
+                continue;
             }
-            if (hw == 0) st_async_b32(peer_pm + b * 512 + h * 4, __float_as_uint(pm), bar);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                mine_nxt[i] = __uint_as_float(kh ? (hw ? r1[16 + i] : r1[i]) : (hw ? r0[16 + i] : r0[i]));
-            pm_nxt = pm;
-            msk_nxt = ((kh ? mhi : mlo) >> (16 * hw)) & 0xFFFFu;
-            return true;
-        };
-        // Stage B of tile u: combine, probabilities, write both copies of this warp's P part.
-        auto stage_b = [&](int u) -> bool {
-            const uint32_t b = u & 1, ph = (u >> 1) & 1;
-            if (!wait_warp(my_sx_full0 + 8 * b, ph, abort, st, 0x2303)) return false;
-            if (arm_thread && u + 2 < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * b, AT_SX_BYTES);
-            float s16[16];
+            // ---- stage B: combine, probabilities, both copies of P ----
+            const uint32_t msk = kh ? mhi : mlo;
+            if (!wait_warp(my_sx_full0 + 8 * xb, xph, abort, st, 0x2303)) { ok = false; break; }
+            if (arm_thread && u + NSX < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * xb, AT_SX_BYTES);
+            float s32[32];
             {
-                const uint8_t* rowp = sx + b * AT_TILE128;
+                const uint8_t* rowp = sx + xb * AT_TILE128;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float4 v = *(const float4*)(rowp + swz(h, 4 * hw + c));
-                    s16[4 * c] = mine_cur[4 * c] + v.x;
-                    s16[4 * c + 1] = mine_cur[4 * c + 1] + v.y;
-                    s16[4 * c + 2] = mine_cur[4 * c + 2] + v.z;
-                    s16[4 * c + 3] = mine_cur[4 * c + 3] + v.w;
+                for (int c = 0; c < 8; ++c) {
+                    const float4 v = *(const float4*)(rowp + swz(h, c));
+                    const float pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        s32[4 * c + e] = __uint_as_float(kh ? r1[4 * c + e] : r0[4 * c + e]) + pv[e];
                 }
             }
-            const float pm_peer = pmx[b * 128 + h];
+            const float pm_peer = pmx[xb * 128 + h];
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * b);
-            // shared running maximum (identical in all four warps of a head), lazy rescale
-            const float mb = (pm_cur == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm_cur + pm_peer) * a.scale_log2;
+            if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * xb);
+            // shared running maximum (identical in both CTAs), lazy rescale
+            const float mb = (pm == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm + pm_peer) * a.scale_log2;
             float alpha = 1.f;
             if (mb > m_used + 8.0f) {
                 alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mb);
                 l *= alpha;
                 m_used = mb;
             }
-            uint32_t pw[8];
+            uint32_t pw[16];
             {
                 float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float p0 = ((msk_cur >> (2 * i)) & 1u) ? ex2(fmaf(s16[2 * i], a.scale_log2, -m_used)) : 0.f;
-                    const float p1 = ((msk_cur >> (2 * i + 1)) & 1u) ? ex2(fmaf(s16[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = ((msk >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
+                    const float p1 = ((msk >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
                     rs0 += p0;
                     rs1 += p1;
                     pw[i] = pack_bf16(p0, p1);
                 }
                 l += rs0 + rs1;
             }
-            // P tile b is free once PV(u-2) is done in both CTAs
-            if (!wait_warp(my_p_free0 + 8 * b, ph ^ 1, abort, st, 0x2304)) return false;
+            // P tile pb is free once PV(u - NPB) is done in both CTAs
+            const uint32_t pb = u % NPB;
+            if (!wait_warp(my_p_free0 + 8 * pb, ((u / NPB) & 1) ^ 1, abort, st, 0x2304)) { ok = false; break; }
             {
-                uint8_t* prow = smem + Lay::OFF_P + b * AT_TILE128;
-                const uint32_t pdst = peer_p + b * AT_TILE128;
-                const uint32_t bar = peer_p_full0 + 8 * b;
+                uint8_t* prow = smem + Lay::OFF_P + pb * AT_TILE128;
+                const uint32_t pdst = peer_p + pb * AT_TILE128;
+                const uint32_t bar = peer_p_full0 + 8 * pb;
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int c = 4 * kh + 2 * hw + q;
+                for (int q = 0; q < 4; ++q) {
+                    const int c = 4 * kh + q;
                     *(uint4*)(prow + swz(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
                     st_async_v4(pdst + swz(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
                 }
             }
             if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                // O may be rescaled only between PV(u-1) and PV(u); this warp owns 128 columns
+                // O may be rescaled only between PV(u-1) and PV(u)
                 const int w = u - 1;
-                if (!wait_warp(my_p_free0 + 8 * (w & 1), (w >> 1) & 1, abort, st, 0x2305)) return false;
+                if (!wait_warp(my_p_free0 + 8 * (w % NPB), (w / NPB) & 1, abort, st, 0x2305)) { ok = false; break; }
                 tc_fence_after();
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t r[32];
-                    const uint32_t ta = tmem + lane_off + TM_O + 128 * hw + c * 32;
+                    const uint32_t ta = tmem + lane_off + TM_O + c * 32;
                     tmem_ld32(ta, r);
                     tmem_wait_ld();
 #pragma unroll
@@ -438,45 +473,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(my_p_full0 + 8 * b);
-            return true;
-        };
-        if (n_tiles > 0) ok = stage_a(0);
-        for (int j = 0; ok && j < n_tiles; ++j) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) mine_cur[i] = mine_nxt[i];
-            pm_cur = pm_nxt;
-            msk_cur = msk_nxt;
-            if (j + 1 < n_tiles && !stage_a(j + 1)) { ok = false; break; }
-            if (!stage_b(j)) { ok = false; break; }
+            if (lane == 0) mbar_arrive(my_p_full0 + 8 * pb);
         }
-        // ---- row sums: this CTA's two partials, then the peer's sum ----
+        // ---- row sums: the B warps combine this CTA's sum with the peer's ----
         float l_tot = 0.f;
-        if (ok && n_tiles > 0) {
-            lx[hw * 128 + h] = l;
+        if (is_b && ok && n_tiles > 0) {
+            // the peer's sum lands in partial-max buffer n_tiles % NSX, free once the
+            // peer has consumed this CTA's partials of tile n_tiles - NSX
+            const uint32_t bf = n_tiles % NSX;
+            ok = wait_warp(my_sx_free0 + 8 * bf, ((n_tiles / NSX) & 1) ^ 1, abort, st, 0x2307);
+            if (ok) st_async_b32(peer_pm + bf * 512 + h * 4, __float_as_uint(l), peer_lx_full);
+            if (ok && wait_warp(smem_u32(&bars->lx_full), 0, abort, st, 0x2308)) l_tot = l + pmx[bf * 128 + h];
+            else ok = false;
+            lx[h] = ok ? l_tot : 0.f;
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->lx_loc));
-            ok = wait_warp(smem_u32(&bars->lx_loc), 0, abort, st, 0x2306);
-            const float l_cta = lx[h] + lx[128 + h];
-            // the peer's sum lands in partial-max buffer n_tiles & 1, free once the
-            // peer has consumed this CTA's partials of tile n_tiles - 2
-            const uint32_t bf = n_tiles & 1;
-            if (ok && hw == 0) {
-                ok = wait_warp(my_sx_free0 + 8 * bf, ((n_tiles >> 1) & 1) ^ 1, abort, st, 0x2307);
-                if (ok) st_async_b32(peer_pm + bf * 512 + h * 4, __float_as_uint(l_cta), peer_lx_full);
-            }
-            if (ok && wait_warp(smem_u32(&bars->lx_full), 0, abort, st, 0x2308)) l_tot = l_cta + pmx[bf * 128 + h];
+        }
+        if (!is_b && n_tiles > 0) {
+            // the A warps take the other half of the epilogue columns
+            if (wait_warp(smem_u32(&bars->lx_loc), 0, abort, st, 0x2306)) l_tot = lx[h];
             else ok = false;
         }
         // ---- epilogue: O / l -> bf16 (this warp's 128 output columns) ----
-        __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + 128 * hw;
-        const bool have_o = ok && n_tiles > 0 && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2307);
+        const int ocol = is_b ? 0 : 128;
+        __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol;
+        const bool have_o = ok && n_tiles > 0 && l_tot > 0.f && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2309);
         if (have_o) tc_fence_after();
-        const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
+        const float inv = have_o ? 1.0f / l_tot : 0.f;
         for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
-            if (have_o) {
-                tmem_ld32(tmem + lane_off + TM_O + 128 * hw + c * 32, r);
+            if (__any_sync(0xffffffffu, have_o)) {
+                tmem_ld32(tmem + lane_off + TM_O + ocol + c * 32, r);
                 tmem_wait_ld();
             }
             uint4* dst = (uint4*)(orow + c * 32);
@@ -494,8 +521,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 dst[i] = w;
             }
         }
-        if (rank == 0 && hw == 0 && a.lse)
-            a.lse[t * 128 + h] = (have_o && l_tot > 0.f) ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        if (rank == 0 && is_b && a.lse)
+            a.lse[t * 128 + h] = have_o ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
     }
     tc_fence_before();
     __syncwarp();
@@ -504,20 +531,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     if (warp == AT_MMA_WARP) tmem_dealloc(tmem, 512);
 }
 
-template <int NST, bool VSEP>
+template <int NST, bool VSEP, int NPB, int NSX>
 static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
-    using Lay = AtLayout<NST, VSEP>;
+    using Lay = AtLayout<NST, VSEP, NPB, NSX>;
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
-    if (cudaFuncSetAttribute(attn_tc_kernel<NST, VSEP>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_tc_kernel<NST, VSEP, NPB, NSX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Lay::SMEM) != cudaSuccess)
         return false;
-    attn_tc_kernel<NST, VSEP><<<(unsigned)(2 * a.total_q), AT_THREADS, Lay::SMEM, s>>>(a);
+    attn_tc_kernel<NST, VSEP, NPB, NSX><<<(unsigned)(2 * a.total_q), AT_THREADS, Lay::SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }
 
+#ifndef DSA_ATTN_NST
+#define DSA_ATTN_NST 3
+#define DSA_ATTN_NPB 2
+#define DSA_ATTN_NSX 1
+#endif
+
 bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s) {
     if (a.total_q <= 0) return true;
-    return a.v_separate ? launch_attn_tc_t<2, true>(a, s) : launch_attn_tc_t<4, false>(a, s);
+    return a.v_separate ? launch_attn_tc_t<2, true, 2, 2>(a, s)
+                        : launch_attn_tc_t<DSA_ATTN_NST, false, DSA_ATTN_NPB, DSA_ATTN_NSX>(a, s);
 }
 
 }  // namespace dsa

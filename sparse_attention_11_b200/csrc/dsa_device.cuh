@@ -107,6 +107,15 @@ DSA_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// Non-blocking probe (test_wait never suspends the thread), for loops that
+// poll several barriers in turn.
+DSA_DEV bool mbar_probe(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
 DSA_DEV bool mbar_test_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
