@@ -21,6 +21,7 @@ cores on a bounded stratified sample of the same workload.
 """
 import argparse
 import datetime
+import hashlib
 import json
 import math
 import os
@@ -178,6 +179,23 @@ def attn_bytes(wl, info):
         wl.total_q * wl.k * 4
 
 
+def captured_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    kernel's sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        tr = json.load(f)
+    h = hashlib.sha256()
+    for rel in tr.get("kernel_sources", []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != tr.get("kernel_sources_sha256"):
+        return None
+    return tr.get(workload, {}).get(kernel)
+
+
 def run_native_workload(wl, steps, warmup, ws_n, rank, sampler=None):
     """Device-timed steps of select + attention on one workload."""
     import torch
@@ -324,13 +342,10 @@ def native(args):
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }
-    traffic = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(traffic):
-        with open(traffic) as f:
-            tr = json.load(f).get(wl.name, {}).get("attn_tc_kernel")
-        if tr:
-            res["roofline"]["traffic"] = tr["bytes_per_launch"]
-            res["roofline"]["traffic_source"] = tr["source"]
+    tr = captured_traffic(wl.name, "attn_tc_kernel")
+    if tr:
+        res["roofline"]["traffic"] = tr["bytes_per_launch"]
+        res["roofline"]["traffic_source"] = tr["source"]
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_native(inp, prob, max(1, min(args.steps, 5)))
         e2e_max = max_over_ranks(e2e_ms, ws_n, dev)
