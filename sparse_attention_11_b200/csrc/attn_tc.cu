@@ -22,8 +22,8 @@
 // two partial maxima of the tile, an upper bound of the true maximum that
 // both form from the exchanged data, with lazy rescaling (moved only when it
 // grows by more than 2^8).  Each CTA writes the bf16 probabilities of its
-// keys into its own P tile and into the peer's (both with st.async), so both
-// hold the full 128 x 64 P (the A operand of O += P V, in shared memory).
+// keys into its own P tile (st.shared) and into the peer's (st.async), so
+// both hold the full 128 x 64 P (the A operand of O += P V, in shared memory).
 // Row sums are combined once at the end.
 //
 // Pipelining.  Stage A (read S, send the partial) and stage B (combine,
@@ -50,6 +50,13 @@
 
 namespace dsa {
 
+// Exchange layout of the partial scores and of P: 16-byte chunk c (4 fp32
+// partials, or 8 bf16 probabilities) of head row h at c*2048 + h*16.  A warp's
+// stores of one chunk then cover 512 contiguous bytes, which the cluster's
+// shared-memory path moves several times faster than 32 scattered 16-byte
+// pieces; for P it is also the no-swizzle K-major operand layout of the MMA
+// (8-row x 16-byte core matrices, 128 B apart along M and 2048 B along K).
+__device__ __forceinline__ uint32_t chunk_off(int h, int c) { return (uint32_t)(c * 2048 + h * 16); }
 constexpr int AT_N = 64;                           // keys per tile
 constexpr uint32_t AT_BLK = AT_N * 128;            // one 64-column block of a tile
 constexpr uint32_t AT_KST = 5 * AT_BLK;            // K part of a stage (max 5 blocks)
@@ -251,7 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                         const uint32_t pb = s_p0 + b * AT_TILE128;
 #pragma unroll
                         for (int ks = 0; ks < AT_N / 16; ++ks)
-                            mma_bf16_ss(tmem + TM_O, sdesc_sw128(pb + ks * 32, 16, 1024),
+                            mma_bf16_ss(tmem + TM_O, sdesc_noswz(pb + ks * 4096, 2048, 128),
                                         sdesc_sw128(vb + ks * 2048, AT_BLK, 1024), idesc_pv, (ju > 0 || ks > 0) ? 1u : 0u);
                         mma_commit(smem_u32(&bars->empty[ju % NST]));
                         mma_commit_mc(smem_u32(&bars->p_free[b]), (uint16_t)3);
@@ -395,7 +402,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
-                    st_async_v4(dst + swz(h, c), w[0], w[1], w[2], w[3], bar);
+                    st_async_v4(dst + chunk_off(h, c), w[0], w[1], w[2], w[3], bar);
                 }
                 st_async_b32(peer_pm + xb * 512 + h * 4, __float_as_uint(pm), bar);
                 continue;
@@ -409,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 const uint8_t* rowp = sx + xb * AT_TILE128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const float4 v = *(const float4*)(rowp + swz(h, c));
+                    const float4 v = *(const float4*)(rowp + chunk_off(h, c));
                     const float pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
@@ -450,8 +457,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int c = 4 * kh + q;
-                    *(uint4*)(prow + swz(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
-                    st_async_v4(pdst + swz(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
+                    *(uint4*)(prow + chunk_off(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
+                    st_async_v4(pdst + chunk_off(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
                 }
             }
             if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {

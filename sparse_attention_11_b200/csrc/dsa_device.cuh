@@ -266,6 +266,18 @@ DSA_DEV uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_by
     return d;
 }
 
+// Shared-memory matrix descriptor, no swizzle (8-row x 16-byte core
+// matrices stored as 128 contiguous bytes).  K-major: lbo = bytes between
+// core matrices along K, sbo = bytes between core matrices along M/N.
+DSA_DEV uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
 // Instruction descriptor, dense, fp32 accumulate.
 //   kind::f16    : a/b format 1 = BF16
 //   kind::f8f6f4 : a/b format 0 = E4M3
