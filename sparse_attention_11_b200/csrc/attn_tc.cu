@@ -14,6 +14,16 @@
 // When V is the latent part of K (V = K[:, :512]) each CTA's V columns are
 // the first 256 of its own K columns, so every gathered byte is used once.
 //
+// Persistence.  The grid holds as many CTA pairs as can be resident at once;
+// pair p takes the queries p, p + P, p + 2P, ...  The K/V stages, S buffers,
+// P tiles and exchange buffers run as rings over the pair's whole sequence of
+// 64-key tiles, across query boundaries, so the gathers and MMAs of one query
+// overlap the start and the end of its neighbours.  Per query the producers
+// publish the index row's validity bits and tile count (a two-slot ring), the
+// softmax warps load the next Q once the last S of the previous query has
+// completed, and the first PV of a query waits until the previous query's
+// epilogue has read O out of tensor memory.
+//
 // Softmax split.  Per 64-key tile each CTA holds a partial S for all 128
 // heads and all 64 keys.  Rank r finishes keys [32r, 32r+32): it sends the
 // other 32 partial columns to its peer and receives the peer's partials of
@@ -24,15 +34,17 @@
 // grows by more than 2^8).  Each CTA writes the bf16 probabilities of its
 // keys into its own P tile (st.shared) and into the peer's (st.async), so
 // both hold the full 128 x 64 P (the A operand of O += P V, in shared memory).
-// Row sums are combined once at the end.
+// Row sums are combined once per query.
 //
 // Pipelining.  Stage A (read S, send the partial) and stage B (combine,
 // probabilities, write P) run in separate warps, so consecutive tiles overlap;
-// the MMA warp issues greedily: PV(u) as soon as P(u) is complete, else S(t)
-// as soon as its K/V stage is full and the S buffer is free.
-// P tiles are double-buffered and released by a tcgen05.commit that arrives
-// on the p_free barrier of both CTAs (PV(t) done in both), so stage B waits
-// for PV(t-2), and for PV(t-1) only when the running maximum moves.
+// the MMA warp issues greedily from two cursors: PV(u) as soon as P(u) is
+// complete, else S(t) as soon as its K/V stage is full and the S buffer is
+// free.  P tiles are double-buffered and released by a tcgen05.commit that
+// arrives on the p_free barrier of both CTAs (PV(t) done in both), so stage B
+// waits for PV(t-2), and for PV(t-1) only when the running maximum moves.
+// The P exchange also keeps the two CTAs within one tile of each other, which
+// the two-arrival p_free barrier relies on.
 //
 // Gathers: seven producer warps copy the selected rows with 16-byte
 // cp.async, 4 rows x 128 bytes per warp instruction, into the
@@ -61,42 +73,53 @@ constexpr int AT_N = 64;                           // keys per tile
 constexpr uint32_t AT_BLK = AT_N * 128;            // one 64-column block of a tile
 constexpr uint32_t AT_KST = 5 * AT_BLK;            // K part of a stage (max 5 blocks)
 constexpr uint32_t AT_VST = 4 * AT_BLK;            // V part (separate V only)
-constexpr uint32_t AT_TILE128 = 128 * 128;         // a 128-row x 128-byte swizzled tile
+constexpr uint32_t AT_TILE128 = 128 * 128;         // a 128-row x 128-byte tile
 constexpr uint32_t AT_SX_BYTES = 128 * 128 + 128 * 4;  // partial scores + partial maxima
 constexpr uint32_t AT_PX_BYTES = 128 * 64;         // the peer's half of P
+constexpr uint32_t AT_LX_BYTES = 128 * 4;          // the peer's row sums
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;  // S: two 64-column buffers
 constexpr int AT_THREADS = 512;  // 7 producer + 1 MMA + 8 softmax warps
 constexpr int AT_PRODUCERS = 7;
 constexpr int AT_MMA_WARP = 7;
-constexpr int AT_SOFT0 = 8;     // first softmax warp (a warpgroup boundary)
+constexpr int AT_SOFT0 = 8;      // first softmax warp (a warpgroup boundary)
+constexpr int AT_SCAN_ROUNDS = (2048 / 32 + AT_PRODUCERS - 1) / AT_PRODUCERS;  // index-row words per producer warp
+constexpr int AT_NTAB = 8;       // tile counts of the queries between the PV and the S cursor
 
-template <int NST, bool VSEP, int NPB = 2, int NSX = 2>
+template <int NST, bool VSEP, int NPB = 2, int NSX = 1>
 struct AtLayout {
     static constexpr uint32_t STAGE = AT_KST + (VSEP ? AT_VST : 0);
-    static constexpr uint32_t OFF_QR = NST * STAGE;           // rank 1's 5th Q block (rope), A of SS MMAs
-    static constexpr uint32_t OFF_P = OFF_QR + AT_TILE128;    // [NPB] P tiles
+    static constexpr uint32_t OFF_QR = NST * STAGE;               // rank 1's 5th Q block (rope), A of SS MMAs
+    static constexpr uint32_t OFF_P = OFF_QR + AT_TILE128;        // [NPB] P tiles
     static constexpr uint32_t OFF_SX = OFF_P + NPB * AT_TILE128;  // [NSX] partial-score tiles
     static constexpr uint32_t OFF_PM = OFF_SX + NSX * AT_TILE128; // [NSX][128] partial maxima
-    static constexpr uint32_t OFF_LX = OFF_PM + NSX * 512;        // [128] row sums for the A warps' epilogue
-    static constexpr uint32_t OFF_VM = OFF_LX + 1024;            // [64] validity bits of 2048 slots
-    static constexpr uint32_t OFF_BAR = OFF_VM + 256;
-    static constexpr uint32_t SMEM = OFF_BAR + 256;
+    static constexpr uint32_t OFF_LX = OFF_PM + NSX * 512;        // [128] combined row sums (B -> A warps)
+    static constexpr uint32_t OFF_LXR = OFF_LX + 512;             // [128] the peer's row sums
+    static constexpr uint32_t OFF_VM = OFF_LXR + 512;             // [2][64] validity bits of 2048 slots
+    static constexpr uint32_t OFF_INFO = OFF_VM + 512;            // [2][8] last used slot per producer warp, [8] tile counts
+    static constexpr uint32_t OFF_BAR = OFF_INFO + 128;
+    static constexpr uint32_t SMEM = OFF_BAR + 512;
 };
 
 struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
-    uint64_t s_full[2], s_empty[2], q_full, o_full;
-    uint64_t p_full[2];   // 4 local B warps + the peer's half of P (bytes)
-    uint64_t p_free[2];   // PV done in both CTAs (multicast commit)
-    uint64_t sx_full[2];  // the peer's partial scores (bytes)
-    uint64_t sx_free[2];  // the peer consumed the partials this CTA sent
-    uint64_t lx_full, lx_loc, drain;
+    uint64_t s_full[2], s_empty[2];
+    uint64_t q_full;         // Q of the next query with tiles is in place (8 softmax warps)
+    uint64_t o_full;         // all PVs of a query done
+    uint64_t o_free;         // its epilogue has read O (8 softmax warps)
+    uint64_t p_full[2];      // 4 local B warps + the peer's half of P (bytes)
+    uint64_t p_free[2];      // PV done in both CTAs (multicast commit)
+    uint64_t sx_full[2];     // the peer's partial scores (bytes)
+    uint64_t sx_free[2];     // the peer consumed the partials this CTA sent
+    uint64_t lx_full;        // the peer's row sums (bytes)
+    uint64_t lx_loc;         // the B warps combined the row sums (for the A warps)
+    uint64_t drain;
+    uint64_t info_full[2];   // query info published (7 producer warps)
+    uint64_t info_empty[2];  // query info consumed (MMA warp + 8 softmax warps)
     uint32_t tmem_base;
     int abort;
-    int max_slot;
 };
-static_assert(sizeof(AtBars) <= 256, "barrier block");
+static_assert(sizeof(AtBars) <= 512, "barrier block");
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 
@@ -104,11 +127,14 @@ template <int NST, bool VSEP, int NPB, int NSX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnTcArgs a) {
     static_assert(AT_SOFT0 % 4 == 0 && AT_PRODUCERS < AT_SOFT0, "warp roles");
+    static_assert(NST >= 1 && NST <= 4 && NPB >= 1 && NPB <= 2 && NSX >= 1 && NSX <= 2, "barrier arrays");
     using Lay = AtLayout<NST, VSEP, NPB, NSX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     AtBars* bars = (AtBars*)(smem + Lay::OFF_BAR);
     uint32_t* vmask = (uint32_t*)(smem + Lay::OFF_VM);
+    int* pmax = (int*)(smem + Lay::OFF_INFO);  // [2][8]
+    int* ntab = pmax + 16;                      // [AT_NTAB]
     if ((uintptr_t)smem != (uintptr_t)smem_raw) {  // the layout needs a 1024-byte aligned base
         if (threadIdx.x == 0) report(a.st, DSA_ERR_UNSUPPORTED, -3);
         return;
@@ -118,16 +144,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     StatusHdr* st = a.st;
     volatile int* abort = &bars->abort;
 
-    const int64_t t = blockIdx.x >> 1;
-    const RowInfo ri = row_info(a.sv, t);
-    if (!ri.ok) {  // both CTAs of the pair take this exit together
-        if (threadIdx.x == 0 && rank == 0) report(st, DSA_ERR_INDEX, t);
-        return;
-    }
+    // queries of this pair: t = pair + i * npairs
+    const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int64_t nq = pair < a.total_q ? (a.total_q - pair + npairs - 1) / npairs : 0;
     const int nb = rank ? 5 : 4;      // 64-column blocks of K held here
     const int col0 = rank ? 256 : 0;  // first K column
     const int dv0 = rank ? 256 : 0;   // first output column
-    const int32_t* irow = a.idx + t * a.ld_idx;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
@@ -137,59 +159,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&bars->s_full[i]), 1);
             mbar_init(smem_u32(&bars->s_empty[i]), 8);  // 4 A + 4 B warps read every S tile
-        }
-        mbar_init(smem_u32(&bars->q_full), 8);
-        mbar_init(smem_u32(&bars->o_full), 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&bars->p_full[i]), 4);  // (only NPB of them are used)
+            mbar_init(smem_u32(&bars->p_full[i]), 4);   // (only NPB of them are used)
             mbar_init(smem_u32(&bars->p_free[i]), 2);
             mbar_init(smem_u32(&bars->sx_full[i]), 1);
             mbar_init(smem_u32(&bars->sx_free[i]), 4);
+            mbar_init(smem_u32(&bars->info_full[i]), AT_PRODUCERS);
+            mbar_init(smem_u32(&bars->info_empty[i]), 9);
         }
+        mbar_init(smem_u32(&bars->q_full), 8);
+        mbar_init(smem_u32(&bars->o_full), 1);
+        mbar_init(smem_u32(&bars->o_free), 8);
         mbar_init(smem_u32(&bars->lx_full), 1);
         mbar_init(smem_u32(&bars->lx_loc), 4);
         mbar_init(smem_u32(&bars->drain), 1);
-        // byte counts of the first phase of every peer-filled barrier
+        // byte counts of the first phase of every peer-filled barrier; each
+        // later phase is armed once the one before it has completed
         for (int i = 0; i < NPB; ++i) mbar_expect_tx(smem_u32(&bars->p_full[i]), AT_PX_BYTES);
-        for (int i = 0; i < NSX; ++i) {
-            mbar_arrive_expect_tx(smem_u32(&bars->sx_full[i]), AT_SX_BYTES);
-        }
-        mbar_arrive_expect_tx(smem_u32(&bars->lx_full), 128 * 4);
+        for (int i = 0; i < NSX; ++i) mbar_arrive_expect_tx(smem_u32(&bars->sx_full[i]), AT_SX_BYTES);
+        mbar_arrive_expect_tx(smem_u32(&bars->lx_full), AT_LX_BYTES);
         bars->abort = 0;
-        bars->max_slot = -1;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < 64; i += blockDim.x) vmask[i] = 0u;
     if (warp == AT_MMA_WARP) tmem_alloc(smem_u32(&bars->tmem_base), 512);
-    // the softmax warps start their Q loads now; they land during the scan
-    uint4 qreg[8] = {};
-    const bool q_loader = warp >= AT_SOFT0;
-    const __nv_bfloat16* qrow = a.q + t * a.q_stride_tok + (int64_t)((warp & 3) * 32 + lane) * a.q_stride_head + col0;
-    if (q_loader) {  // block (warp - 3) >> 2 of this head's Q half
-        const uint4* src = (const uint4*)(qrow + 64 * (((int)warp - AT_SOFT0) >> 2));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qreg[i] = __ldg(src + i);
-    }
-    __syncthreads();
-    // validity bits of the index row and the number of 64-slot tiles (up to
-    // the last valid slot)
-    {
-        int m = -1;
-        for (int j0 = (int)(warp * 32); j0 < a.k_sel; j0 += (int)blockDim.x) {
-            const int j = j0 + (int)lane;
-            const int32_t v = j < a.k_sel ? __ldg(irow + j) : -1;
-            const uint32_t bits = __ballot_sync(0xffffffffu, v >= 0 && v < ri.seqlen_k);
-            if (v >= 0) m = j;
-            if (lane == 0 && j0 < 2048) vmask[j0 >> 5] = bits;
-        }
-        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0 && m >= 0) atomicMax(&bars->max_slot, m);
-    }
     tc_fence_before();
-    cluster_sync();  // barriers of both CTAs initialised and armed; max_slot final
+    cluster_sync();  // barriers of both CTAs initialised and armed
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const int n_tiles = (bars->max_slot + AT_N) / AT_N;
 
     const uint32_t s_stage0 = smem_u32(smem);
     const uint32_t s_p0 = smem_u32(smem + Lay::OFF_P);
@@ -200,40 +195,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         // 16 groups of 4 keys per tile; warp w takes groups w, w+7, w+14
         const int sub = (int)(lane >> 3), chunk = (int)(lane & 7);
         const int ngrp = (16 - (int)warp + AT_PRODUCERS - 1) / AT_PRODUCERS;
-        int32_t nxt[3] = {-1, -1, -1};
-        auto load_idx = [&](int j) {
-#pragma unroll
-            for (int gi = 0; gi < 3; ++gi) {
-                const int slot = j * AT_N + 4 * ((int)warp + AT_PRODUCERS * gi) + sub;
-                nxt[gi] = (gi < ngrp && slot < a.k_sel) ? __ldg(irow + slot) : -1;
+        uint32_t g = 0;  // tile of the pair's whole sequence
+        bool ok = true;
+        for (int64_t qi = 0; ok && qi < nq; ++qi) {
+            const int64_t t = pair + qi * npairs;
+            const RowInfo ri = row_info(a.sv, t);
+            const int32_t* irow = a.idx + t * a.ld_idx;
+            const uint32_t slot = (uint32_t)(qi & 1);
+            // ---- query info: validity bits of the index row, last used slot ----
+            if (!wait_warp(smem_u32(&bars->info_empty[slot]), (uint32_t)((qi >> 1) & 1) ^ 1u, abort, st, 0x2102)) {
+                ok = false;
+                break;
             }
-        };
-        if (n_tiles > 0) load_idx(0);
-        for (int j = 0; j < n_tiles; ++j) {
-            const uint32_t s = j % NST;
-            int32_t cur[3];
+            int m = -1;
+            {
+                int32_t v[AT_SCAN_ROUNDS];
 #pragma unroll
-            for (int gi = 0; gi < 3; ++gi) cur[gi] = nxt[gi];
-            if (j + 1 < n_tiles) load_idx(j + 1);
-            if (!wait_warp(smem_u32(&bars->empty[s]), ((j / NST) & 1) ^ 1, abort, st, 0x2101)) break;
-            const uint32_t kst = s_stage0 + s * Lay::STAGE;
-#pragma unroll
-            for (int gi = 0; gi < 3; ++gi) {
-                if (gi >= ngrp) break;
-                const int32_t v = cur[gi];
-                if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
-                const int64_t r = ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0);
-                const int key = 4 * ((int)warp + AT_PRODUCERS * gi) + sub;  // key of the tile
-                const __nv_bfloat16* src = a.k + r * a.k_stride + col0 + chunk * 8;
-                const uint32_t dst = kst + swz(key, chunk);
-                for (int kb = 0; kb < nb; ++kb) cp_async16(dst + kb * AT_BLK, src + kb * 64);
-                if (VSEP) {
-                    const __nv_bfloat16* vs = a.v + r * a.v_stride + dv0 + chunk * 8;
-#pragma unroll
-                    for (int vb = 0; vb < 4; ++vb) cp_async16(dst + AT_KST + vb * AT_BLK, vs + vb * 64);
+                for (int r = 0; r < AT_SCAN_ROUNDS; ++r) {
+                    const int j = ((int)warp + AT_PRODUCERS * r) * 32 + (int)lane;
+                    v[r] = (ri.ok && j < a.k_sel) ? __ldg(irow + j) : -1;
                 }
+#pragma unroll
+                for (int r = 0; r < AT_SCAN_ROUNDS; ++r) {
+                    const int w = (int)warp + AT_PRODUCERS * r;  // 32-slot word of the row
+                    const uint32_t bits = __ballot_sync(0xffffffffu, v[r] >= 0 && v[r] < ri.seqlen_k);
+                    if (v[r] >= 0) m = w * 32 + (int)lane;
+                    if (lane == 0 && w < 64) vmask[slot * 64 + w] = bits;
+                }
+                for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             }
-            cp_async_arrive(smem_u32(&bars->full[s]));
+            if (!ri.ok && warp == 0 && lane == 0 && rank == 0) report(st, DSA_ERR_INDEX, t);
+            if (lane == 0) {
+                pmax[slot * 8 + warp] = m;
+                mbar_arrive(smem_u32(&bars->info_full[slot]));
+            }
+            if (!wait_warp(smem_u32(&bars->info_full[slot]), (uint32_t)((qi >> 1) & 1), abort, st, 0x2103)) {
+                ok = false;
+                break;
+            }
+            int mx = -1;
+#pragma unroll
+            for (int w = 0; w < AT_PRODUCERS; ++w) mx = max(mx, pmax[slot * 8 + w]);
+            const int n_tiles = (mx + AT_N) / AT_N;
+            // ---- the query's tiles ----
+            int32_t nxt[3] = {-1, -1, -1};
+            auto load_idx = [&](int j) {
+#pragma unroll
+                for (int gi = 0; gi < 3; ++gi) {
+                    const int sj = j * AT_N + 4 * ((int)warp + AT_PRODUCERS * gi) + sub;
+                    nxt[gi] = (gi < ngrp && sj < a.k_sel) ? __ldg(irow + sj) : -1;
+                }
+            };
+            if (n_tiles > 0) load_idx(0);
+            for (int j = 0; j < n_tiles; ++j, ++g) {
+                const uint32_t s = g % NST;
+                int32_t cur[3];
+#pragma unroll
+                for (int gi = 0; gi < 3; ++gi) cur[gi] = nxt[gi];
+                if (j + 1 < n_tiles) load_idx(j + 1);
+                if (!wait_warp(smem_u32(&bars->empty[s]), ((g / NST) & 1) ^ 1, abort, st, 0x2101)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t kst = s_stage0 + s * Lay::STAGE;
+#pragma unroll
+                for (int gi = 0; gi < 3; ++gi) {
+                    if (gi >= ngrp) break;
+                    const int32_t v = cur[gi];
+                    if (v >= ri.seqlen_k) report(st, DSA_ERR_INDEX, t);
+                    const int64_t r = ri.key_base + ((v >= 0 && v < ri.seqlen_k) ? v : 0);
+                    const int key = 4 * ((int)warp + AT_PRODUCERS * gi) + sub;  // key of the tile
+                    const __nv_bfloat16* src = a.k + r * a.k_stride + col0 + chunk * 8;
+                    const uint32_t dst = kst + swz(key, chunk);
+                    for (int kb = 0; kb < nb; ++kb) cp_async16(dst + kb * AT_BLK, src + kb * 64);
+                    if (VSEP) {
+                        const __nv_bfloat16* vs = a.v + r * a.v_stride + dv0 + chunk * 8;
+#pragma unroll
+                        for (int vb = 0; vb < 4; ++vb) cp_async16(dst + AT_KST + vb * AT_BLK, vs + vb * 64);
+                    }
+                }
+                cp_async_arrive(smem_u32(&bars->full[s]));
+            }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == AT_MMA_WARP) {
@@ -241,58 +283,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
         constexpr uint32_t idesc_s = idesc_make(1, 1, false, 128, AT_N);
         constexpr uint32_t idesc_pv = idesc_make(1, 1, true, 128, 256);
-        bool ok = n_tiles > 0 && wait_warp(smem_u32(&bars->q_full), 0, abort, st, 0x2201);
-        // Greedy issue: PV(ju) as soon as its P tile is complete (ju < js), else
-        // S(js) as soon as its K/V stage is full and the S buffer is free.
-        int js = 0, ju = 0;
+        // Two cursors over the pair's tile sequence.  S cursor: query qs (ns
+        // tiles once its info is read, else -1), tile js, sequence tile gs,
+        // nqs queries with tiles begun.  PV cursor: query-with-tiles nqu, tile
+        // ju, sequence tile gu; tile counts of begun queries are kept in ntab.
+        int64_t qs = 0;
+        int js = 0, ns = -1, ju = 0;
+        uint32_t gs = 0, nqs = 0, gu = 0, nqu = 0;
+        bool ok = true;
         long long idle0 = clock64();
-        while (ok && ju < n_tiles) {
+        while (ok && (qs < nq || nqu < nqs)) {
             bool done = false;
-            if (ju < js) {
-                const uint32_t b = ju % NPB;
-                if (__all_sync(0xffffffffu, mbar_probe(smem_u32(&bars->p_full[b]), (ju / NPB) & 1))) {
+            // ---- PV cursor (S(gu) issued, so its query has begun) ----
+            if (gu < gs) {
+                const int nu = ntab[nqu % AT_NTAB];
+                const uint32_t b = gu % NPB;
+                bool rdy = mbar_probe(smem_u32(&bars->p_full[b]), (gu / NPB) & 1);
+                if (ju == 0 && nqu > 0) rdy = rdy && mbar_probe(smem_u32(&bars->o_free), (nqu - 1) & 1);
+                if (__all_sync(0xffffffffu, rdy)) {
                     tc_fence_after();
                     if (lane == 0) {
-                        if (ju + NPB < n_tiles) mbar_expect_tx(smem_u32(&bars->p_full[b]), AT_PX_BYTES);
-                        const uint32_t vb = s_stage0 + (ju % NST) * Lay::STAGE + (VSEP ? AT_KST : 0);
+                        mbar_expect_tx(smem_u32(&bars->p_full[b]), AT_PX_BYTES);  // its next phase
+                        const uint32_t vb = s_stage0 + (gu % NST) * Lay::STAGE + (VSEP ? AT_KST : 0);
                         const uint32_t pb = s_p0 + b * AT_TILE128;
 #pragma unroll
                         for (int ks = 0; ks < AT_N / 16; ++ks)
                             mma_bf16_ss(tmem + TM_O, sdesc_noswz(pb + ks * 4096, 2048, 128),
                                         sdesc_sw128(vb + ks * 2048, AT_BLK, 1024), idesc_pv, (ju > 0 || ks > 0) ? 1u : 0u);
-                        mma_commit(smem_u32(&bars->empty[ju % NST]));
+                        mma_commit(smem_u32(&bars->empty[gu % NST]));
                         mma_commit_mc(smem_u32(&bars->p_free[b]), (uint16_t)3);
+                        if (ju + 1 == nu) mma_commit(smem_u32(&bars->o_full));
                     }
                     __syncwarp();
-                    ++ju;
+                    ++gu;
+                    if (++ju == nu) {
+                        ju = 0;
+                        ++nqu;
+                    }
                     done = true;
                 }
             }
-            if (!done && js < n_tiles) {
-                const uint32_t s = js % NST, sb = js & 1;
-                const bool rdy = mbar_probe(smem_u32(&bars->full[s]), (js / NST) & 1) &&
-                                 mbar_probe(smem_u32(&bars->s_empty[sb]), ((js >> 1) & 1) ^ 1);
-                if (__all_sync(0xffffffffu, rdy)) {
-                    fence_proxy_async();
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t kst = s_stage0 + s * Lay::STAGE;
-                        const uint32_t d = tmem + TM_S + 64 * sb;
-                        for (int kb = 0; kb < 4; ++kb)
+            // ---- S cursor ----
+            if (!done && qs < nq) {
+                if (ns < 0) {
+                    const uint32_t slot = (uint32_t)(qs & 1);
+                    if (__all_sync(0xffffffffu, mbar_probe(smem_u32(&bars->info_full[slot]), (uint32_t)((qs >> 1) & 1)))) {
+                        int mx = -1;
 #pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                mma_bf16_ts(d, tmem + TM_Q + kb * 32 + ks * 8, sdesc_sw128(kst + kb * AT_BLK + ks * 32, 16, 1024),
-                                            idesc_s, (kb | ks) ? 1u : 0u);
-                        if (nb == 5)  // the rope block: Q from shared memory
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                mma_bf16_ss(d, sdesc_sw128(s_qr + ks * 32, 16, 1024),
-                                            sdesc_sw128(kst + 4 * AT_BLK + ks * 32, 16, 1024), idesc_s, 1u);
-                        mma_commit(smem_u32(&bars->s_full[sb]));
+                        for (int w = 0; w < AT_PRODUCERS; ++w) mx = max(mx, pmax[slot * 8 + w]);
+                        ns = (mx + AT_N) / AT_N;
+                        if (lane == 0) {
+                            if (ns > 0) ntab[nqs % AT_NTAB] = ns;
+                            mbar_arrive(smem_u32(&bars->info_empty[slot]));
+                        }
+                        __syncwarp();
+                        if (ns == 0) {
+                            ns = -1;
+                            ++qs;
+                        }
+                        done = true;
                     }
-                    __syncwarp();
-                    ++js;
-                    done = true;
+                } else {
+                    const uint32_t s = gs % NST, sb = gs & 1;
+                    bool rdy = mbar_probe(smem_u32(&bars->full[s]), (gs / NST) & 1) &&
+                               mbar_probe(smem_u32(&bars->s_empty[sb]), ((gs >> 1) & 1) ^ 1);
+                    if (js == 0) rdy = rdy && mbar_probe(smem_u32(&bars->q_full), nqs & 1);
+                    if (__all_sync(0xffffffffu, rdy)) {
+                        fence_proxy_async();
+                        tc_fence_after();
+                        if (lane == 0) {
+                            const uint32_t kst = s_stage0 + s * Lay::STAGE;
+                            const uint32_t d = tmem + TM_S + 64 * sb;
+                            for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    mma_bf16_ts(d, tmem + TM_Q + kb * 32 + ks * 8,
+                                                sdesc_sw128(kst + kb * AT_BLK + ks * 32, 16, 1024), idesc_s,
+                                                (kb | ks) ? 1u : 0u);
+                            if (nb == 5)  // the rope block: Q from shared memory
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    mma_bf16_ss(d, sdesc_sw128(s_qr + ks * 32, 16, 1024),
+                                                sdesc_sw128(kst + 4 * AT_BLK + ks * 32, 16, 1024), idesc_s, 1u);
+                            mma_commit(smem_u32(&bars->s_full[sb]));
+                        }
+                        __syncwarp();
+                        ++gs;
+                        if (++js == ns) {
+                            js = 0;
+                            ns = -1;
+                            ++qs;
+                            ++nqs;
+                        }
+                        done = true;
+                    }
                 }
             }
             if (done) {
@@ -311,7 +395,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 }
             }
         }
-        if (ok && n_tiles > 0 && lane == 0) mma_commit(smem_u32(&bars->o_full));
         if (*abort && lane == 0) {
             mma_commit(smem_u32(&bars->drain));
             mbar_wait(smem_u32(&bars->drain), 0, nullptr, st, 0x2205, 1ll << 28);
@@ -323,6 +406,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         // partial columns; warps 12..15 ("B") read their own 32 columns of the
         // same tile, combine them with the peer's partials, form the
         // probabilities and write P.  Both groups run every tile concurrently.
+        // Per query: load Q (after the previous query's last S), finish the
+        // previous query (row sums, O / l), then the tiles.
         asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
         const uint32_t quad = warp & 3;
         const bool is_b = warp >= AT_SOFT0 + 4;
@@ -332,8 +417,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         uint8_t* sx = smem + Lay::OFF_SX;
         const float* pmx = (const float*)(smem + Lay::OFF_PM);
         float* lx = (float*)(smem + Lay::OFF_LX);
+        const float* lxr = (const float*)(smem + Lay::OFF_LXR);
         const uint32_t peer_sx = mapa(smem_u32(sx), peer);
         const uint32_t peer_pm = mapa(smem_u32(smem + Lay::OFF_PM), peer);
+        const uint32_t peer_lxr = mapa(smem_u32(smem + Lay::OFF_LXR), peer);
         const uint32_t peer_p = mapa(s_p0, peer);
         const uint32_t peer_sx_full0 = mapa(smem_u32(&bars->sx_full[0]), peer);
         const uint32_t peer_sx_free0 = mapa(smem_u32(&bars->sx_free[0]), peer);
@@ -342,200 +429,282 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         const uint32_t my_sx_full0 = smem_u32(&bars->sx_full[0]), my_sx_free0 = smem_u32(&bars->sx_free[0]);
         const uint32_t my_p_full0 = smem_u32(&bars->p_full[0]), my_p_free0 = smem_u32(&bars->p_free[0]);
         const bool arm_thread = threadIdx.x == (AT_SOFT0 + 4) * 32;
-        float m_used = -INFINITY, l = 0.f;
-        bool ok = true;
-        if (n_tiles > 0) {
-            // ---- Q half -> TMEM (A operand of S = Q K^T); the A and B warps of a
-            // quadrant take alternate 64-column blocks, block (is_b) was loaded early ----
-            for (int kb = is_b ? 1 : 0; kb < nb; kb += 2) {
-                uint32_t r[32];
-                if (kb > 1) {
-                    const uint4* src = (const uint4*)(qrow + kb * 64);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) qreg[i] = __ldg(src + i);
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    r[4 * i] = qreg[i].x; r[4 * i + 1] = qreg[i].y; r[4 * i + 2] = qreg[i].z; r[4 * i + 3] = qreg[i].w;
-                }
-                if (kb < 4) {
-                    tmem_st32(tmem + lane_off + TM_Q + kb * 32, r);
-                } else {
-                    uint8_t* qr = smem + Lay::OFF_QR;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *(uint4*)(qr + swz(h, c)) = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
-                }
+        const int ocol = is_b ? 0 : 128;  // this warp's 128 of the CTA's 256 output columns
+
+        // Row sums, O / l -> bf16 and lse of query t, the e-th query with tiles.
+        auto epilogue = [&](int64_t t, uint32_t e, float m_used, float l) -> bool {
+            float l_tot = 0.f;
+            if (is_b) {
+                // the peer's buffer is free: it read its previous sums before its
+                // A warps sent the partials of this query's tiles
+                st_async_b32(peer_lxr + h * 4, __float_as_uint(l), peer_lx_full);
+                if (!wait_warp(smem_u32(&bars->lx_full), e & 1, abort, st, 0x2308)) return false;
+                l_tot = l + lxr[h];
+                if (arm_thread) mbar_arrive_expect_tx(smem_u32(&bars->lx_full), AT_LX_BYTES);  // its next phase
+                lx[h] = l_tot;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->lx_loc));
+            } else {
+                if (!wait_warp(smem_u32(&bars->lx_loc), e & 1, abort, st, 0x2306)) return false;
+                l_tot = lx[h];
             }
-            tmem_wait_st();
-            fence_proxy_async();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
-        }
-        for (int u = 0; ok && u < n_tiles; ++u) {
-            const uint32_t b = u & 1, ph = (u >> 1) & 1;  // S buffer and its phase
-            const uint32_t xb = u % NSX, xph = (u / NSX) & 1;  // partial-score buffer and its phase
-            const uint32_t mlo = u < 32 ? vmask[2 * u] : 0u, mhi = u < 32 ? vmask[2 * u + 1] : 0u;
-            if (!wait_warp(smem_u32(&bars->s_full[b]), ph, abort, st, 0x2301)) { ok = false; break; }
+            if (!wait_warp(smem_u32(&bars->o_full), e & 1, abort, st, 0x2309)) return false;
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            tmem_ld32(tmem + lane_off + TM_S + 64 * b, r0);
-            tmem_ld32(tmem + lane_off + TM_S + 64 * b + 32, r1);
+            const bool have_o = l_tot > 0.f;
+            const float inv = have_o ? 1.0f / l_tot : 0.f;
+            __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol;
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + TM_O + ocol + c * 32, r[c]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b]));
-            float pm = -INFINITY;  // partial maximum of this CTA's row over the tile's valid keys
+            if (lane == 0) mbar_arrive(smem_u32(&bars->o_free));  // O may be overwritten now
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if ((mlo >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r0[i]));
-                if ((mhi >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r1[i]));
-            }
-            if (!is_b) {
-                // ---- stage A: send the peer's 32 partial columns and the partial max ----
-                if (!wait_warp(my_sx_free0 + 8 * xb, xph ^ 1, abort, st, 0x2302)) { ok = false; break; }
-                const uint32_t dst = peer_sx + xb * AT_TILE128;
-                const uint32_t bar = peer_sx_full0 + 8 * xb;
+            for (int c = 0; c < 4; ++c) {
+                uint4* dst = (uint4*)(orow + c * 32);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {  // the peer's keys: [32,64) for rank 0, [0,32) for rank 1
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
-                    st_async_v4(dst + chunk_off(h, c), w[0], w[1], w[2], w[3], bar);
+                for (int i = 0; i < 4; ++i) {
+                    uint4 w;
+                    w.x = pack_bf16(__uint_as_float(r[c][8 * i + 0]) * inv, __uint_as_float(r[c][8 * i + 1]) * inv);
+                    w.y = pack_bf16(__uint_as_float(r[c][8 * i + 2]) * inv, __uint_as_float(r[c][8 * i + 3]) * inv);
+                    w.z = pack_bf16(__uint_as_float(r[c][8 * i + 4]) * inv, __uint_as_float(r[c][8 * i + 5]) * inv);
+                    w.w = pack_bf16(__uint_as_float(r[c][8 * i + 6]) * inv, __uint_as_float(r[c][8 * i + 7]) * inv);
+                    dst[i] = w;
                 }
-                st_async_b32(peer_pm + xb * 512 + h * 4, __float_as_uint(pm), bar);
+            }
+            if (rank == 0 && is_b && a.lse)
+                a.lse[t * 128 + h] = have_o ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+            return true;
+        };
+
+        uint32_t g = 0;    // tile of the pair's whole sequence
+        uint32_t nqt = 0;  // queries with tiles begun
+        bool ok = true;
+        bool pend = false;  // a query's epilogue is still to be done
+        int64_t t_pend = 0;
+        float m_pend = -INFINITY, l_pend = 0.f;
+        for (int64_t qi = 0; ok && qi < nq; ++qi) {
+            const int64_t t = pair + qi * npairs;
+            const uint32_t slot = (uint32_t)(qi & 1);
+            if (!wait_warp(smem_u32(&bars->info_full[slot]), (uint32_t)((qi >> 1) & 1), abort, st, 0x2310)) {
+                ok = false;
+                break;
+            }
+            int mx = -1;
+#pragma unroll
+            for (int w = 0; w < AT_PRODUCERS; ++w) mx = max(mx, pmax[slot * 8 + w]);
+            const int n_tiles = (mx + AT_N) / AT_N;
+            if (n_tiles == 0) {  // nothing selected: zero rows, lse -inf
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->info_empty[slot]));
+                uint4* dst = (uint4*)(a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (rank == 0 && is_b && a.lse) a.lse[t * 128 + h] = -INFINITY;
                 continue;
             }
-            // ---- stage B: combine, probabilities, both copies of P ----
-            const uint32_t msk = kh ? mhi : mlo;
-            if (!wait_warp(my_sx_full0 + 8 * xb, xph, abort, st, 0x2303)) { ok = false; break; }
-            if (arm_thread && u + NSX < n_tiles) mbar_arrive_expect_tx(my_sx_full0 + 8 * xb, AT_SX_BYTES);
-            float s32[32];
+            // ---- Q of this query -> TMEM (A operand of S = Q K^T); every S of the
+            // earlier queries has completed (this warp saw its s_full) ----
             {
-                const uint8_t* rowp = sx + xb * AT_TILE128;
+                const __nv_bfloat16* qrow = a.q + t * a.q_stride_tok + (int64_t)h * a.q_stride_head + col0;
+                uint4 qreg[3][8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 v = *(const float4*)(rowp + chunk_off(h, c));
-                    const float pv[4] = {v.x, v.y, v.z, v.w};
+                for (int i = 0; i < 3; ++i) {
+                    const int kb = 2 * i + (is_b ? 1 : 0);
+                    if (kb < nb) {
+                        const uint4* src = (const uint4*)(qrow + kb * 64);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        s32[4 * c + e] = __uint_as_float(kh ? r1[4 * c + e] : r0[4 * c + e]) + pv[e];
+                        for (int j = 0; j < 8; ++j) qreg[i][j] = __ldg(src + j);
+                    }
                 }
-            }
-            const float pm_peer = pmx[xb * 128 + h];
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * xb);
-            // shared running maximum (identical in both CTAs), lazy rescale
-            const float mb = (pm == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm + pm_peer) * a.scale_log2;
-            float alpha = 1.f;
-            if (mb > m_used + 8.0f) {
-                alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mb);
-                l *= alpha;
-                m_used = mb;
-            }
-            uint32_t pw[16];
-            {
-                float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = ((msk >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
-                    const float p1 = ((msk >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
-                    rs0 += p0;
-                    rs1 += p1;
-                    pw[i] = pack_bf16(p0, p1);
-                }
-                l += rs0 + rs1;
-            }
-            // P tile pb is free once PV(u - NPB) is done in both CTAs
-            const uint32_t pb = u % NPB;
-            if (!wait_warp(my_p_free0 + 8 * pb, ((u / NPB) & 1) ^ 1, abort, st, 0x2304)) { ok = false; break; }
-            {
-                uint8_t* prow = smem + Lay::OFF_P + pb * AT_TILE128;
-                const uint32_t pdst = peer_p + pb * AT_TILE128;
-                const uint32_t bar = peer_p_full0 + 8 * pb;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = 4 * kh + q;
-                    *(uint4*)(prow + chunk_off(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
-                    st_async_v4(pdst + chunk_off(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
-                }
-            }
-            if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                // O may be rescaled only between PV(u-1) and PV(u)
-                const int w = u - 1;
-                if (!wait_warp(my_p_free0 + 8 * (w % NPB), (w / NPB) & 1, abort, st, 0x2305)) { ok = false; break; }
-                tc_fence_after();
-                for (int c = 0; c < 8; ++c) {
+                for (int i = 0; i < 3; ++i) {
+                    const int kb = 2 * i + (is_b ? 1 : 0);
+                    if (kb >= nb) continue;
                     uint32_t r[32];
-                    const uint32_t ta = tmem + lane_off + TM_O + c * 32;
-                    tmem_ld32(ta, r);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(ta, r);
+                    for (int j = 0; j < 8; ++j) {
+                        r[4 * j] = qreg[i][j].x;
+                        r[4 * j + 1] = qreg[i][j].y;
+                        r[4 * j + 2] = qreg[i][j].z;
+                        r[4 * j + 3] = qreg[i][j].w;
+                    }
+                    if (kb < 4) {
+                        tmem_st32(tmem + lane_off + TM_Q + kb * 32, r);
+                    } else {
+                        uint8_t* qr = smem + Lay::OFF_QR;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *(uint4*)(qr + swz(h, c)) = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+                    }
                 }
                 tmem_wait_st();
+                fence_proxy_async();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->q_full));
             }
-            fence_proxy_async();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(my_p_full0 + 8 * pb);
-        }
-        // ---- row sums: the B warps combine this CTA's sum with the peer's ----
-        float l_tot = 0.f;
-        if (is_b && ok && n_tiles > 0) {
-            // the peer's sum lands in partial-max buffer n_tiles % NSX, free once the
-            // peer has consumed this CTA's partials of tile n_tiles - NSX
-            const uint32_t bf = n_tiles % NSX;
-            ok = wait_warp(my_sx_free0 + 8 * bf, ((n_tiles / NSX) & 1) ^ 1, abort, st, 0x2307);
-            if (ok) st_async_b32(peer_pm + bf * 512 + h * 4, __float_as_uint(l), peer_lx_full);
-            if (ok && wait_warp(smem_u32(&bars->lx_full), 0, abort, st, 0x2308)) l_tot = l + pmx[bf * 128 + h];
-            else ok = false;
-            lx[h] = ok ? l_tot : 0.f;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars->lx_loc));
-        }
-        if (!is_b && n_tiles > 0) {
-            // the A warps take the other half of the epilogue columns
-            if (wait_warp(smem_u32(&bars->lx_loc), 0, abort, st, 0x2306)) l_tot = lx[h];
-            else ok = false;
-        }
-        // ---- epilogue: O / l -> bf16 (this warp's 128 output columns) ----
-        const int ocol = is_b ? 0 : 128;
-        __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol;
-        const bool have_o = ok && n_tiles > 0 && l_tot > 0.f && wait_warp(smem_u32(&bars->o_full), 0, abort, st, 0x2309);
-        if (have_o) tc_fence_after();
-        const float inv = have_o ? 1.0f / l_tot : 0.f;
-        for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            if (__any_sync(0xffffffffu, have_o)) {
-                tmem_ld32(tmem + lane_off + TM_O + ocol + c * 32, r);
-                tmem_wait_ld();
-            }
-            uint4* dst = (uint4*)(orow + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint4 w;
-                if (have_o) {
-                    w.x = pack_bf16(__uint_as_float(r[8 * i + 0]) * inv, __uint_as_float(r[8 * i + 1]) * inv);
-                    w.y = pack_bf16(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv);
-                    w.z = pack_bf16(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv);
-                    w.w = pack_bf16(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv);
-                } else {
-                    w = make_uint4(0u, 0u, 0u, 0u);
+            // ---- the previous query's epilogue (this query's first S overlap it) ----
+            if (pend) {
+                if (!epilogue(t_pend, nqt - 1, m_pend, l_pend)) {
+                    ok = false;
+                    break;
                 }
-                dst[i] = w;
+                pend = false;
             }
+            float m_used = -INFINITY, l = 0.f;
+            for (int u = 0; ok && u < n_tiles; ++u, ++g) {
+                const uint32_t b = g & 1, ph = (g >> 1) & 1;          // S buffer and its phase
+                const uint32_t xb = g % NSX, xph = (g / NSX) & 1;      // partial-score buffer and its phase
+                const uint32_t mlo = vmask[slot * 64 + 2 * u], mhi = vmask[slot * 64 + 2 * u + 1];
+                if (!wait_warp(smem_u32(&bars->s_full[b]), ph, abort, st, 0x2301)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + TM_S + 64 * b, r0);
+                tmem_ld32(tmem + lane_off + TM_S + 64 * b + 32, r1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b]));
+                float pm = -INFINITY;  // partial maximum of this CTA's row over the tile's valid keys
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if ((mlo >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r0[i]));
+                    if ((mhi >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r1[i]));
+                }
+                if (!is_b) {
+                    // ---- stage A: send the peer's 32 partial columns and the partial max ----
+                    if (!wait_warp(my_sx_free0 + 8 * xb, xph ^ 1, abort, st, 0x2302)) { ok = false; break; }
+                    const uint32_t dst = peer_sx + xb * AT_TILE128;
+                    const uint32_t bar = peer_sx_full0 + 8 * xb;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {  // the peer's keys: [32,64) for rank 0, [0,32) for rank 1
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
+                        st_async_v4(dst + chunk_off(h, c), w[0], w[1], w[2], w[3], bar);
+                    }
+                    st_async_b32(peer_pm + xb * 512 + h * 4, __float_as_uint(pm), bar);
+                    continue;
+                }
+                // ---- stage B: combine, probabilities, both copies of P ----
+                const uint32_t msk = kh ? mhi : mlo;
+                if (!wait_warp(my_sx_full0 + 8 * xb, xph, abort, st, 0x2303)) { ok = false; break; }
+                if (arm_thread) mbar_arrive_expect_tx(my_sx_full0 + 8 * xb, AT_SX_BYTES);  // its next phase
+                float s32[32];
+                {
+                    const uint8_t* rowp = sx + xb * AT_TILE128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 v = *(const float4*)(rowp + chunk_off(h, c));
+                        const float pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            s32[4 * c + e] = __uint_as_float(kh ? r1[4 * c + e] : r0[4 * c + e]) + pv[e];
+                    }
+                }
+                const float pm_peer = pmx[xb * 128 + h];
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(peer_sx_free0 + 8 * xb);
+                // shared running maximum (identical in both CTAs), lazy rescale
+                const float mb = (pm == -INFINITY || pm_peer == -INFINITY) ? -INFINITY : (pm + pm_peer) * a.scale_log2;
+                float alpha = 1.f;
+                if (mb > m_used + 8.0f) {
+                    alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mb);
+                    l *= alpha;
+                    m_used = mb;
+                }
+                uint32_t pw[16];
+                {
+                    float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = ((msk >> (2 * i)) & 1u) ? ex2(fmaf(s32[2 * i], a.scale_log2, -m_used)) : 0.f;
+                        const float p1 = ((msk >> (2 * i + 1)) & 1u) ? ex2(fmaf(s32[2 * i + 1], a.scale_log2, -m_used)) : 0.f;
+                        rs0 += p0;
+                        rs1 += p1;
+                        pw[i] = pack_bf16(p0, p1);
+                    }
+                    l += rs0 + rs1;
+                }
+                // P tile pb is free once PV(g - NPB) is done in both CTAs
+                const uint32_t pb = g % NPB;
+                if (!wait_warp(my_p_free0 + 8 * pb, ((g / NPB) & 1) ^ 1, abort, st, 0x2304)) { ok = false; break; }
+                {
+                    uint8_t* prow = smem + Lay::OFF_P + pb * AT_TILE128;
+                    const uint32_t pdst = peer_p + pb * AT_TILE128;
+                    const uint32_t bar = peer_p_full0 + 8 * pb;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int c = 4 * kh + q;
+                        *(uint4*)(prow + chunk_off(h, c)) = make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
+                        st_async_v4(pdst + chunk_off(h, c), pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3], bar);
+                    }
+                }
+                if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O may be rescaled only between PV(g-1) and PV(g)
+                    const uint32_t w = g - 1;
+                    if (!wait_warp(my_p_free0 + 8 * (w % NPB), (w / NPB) & 1, abort, st, 0x2305)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t r[32];
+                        const uint32_t ta = tmem + lane_off + TM_O + c * 32;
+                        tmem_ld32(ta, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st32(ta, r);
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(my_p_full0 + 8 * pb);
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->info_empty[slot]));
+            pend = true;
+            t_pend = t;
+            m_pend = m_used;
+            l_pend = l;
+            ++nqt;
         }
-        if (rank == 0 && is_b && a.lse)
-            a.lse[t * 128 + h] = have_o ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        if (ok && pend) ok = epilogue(t_pend, nqt - 1, m_pend, l_pend);
     }
     tc_fence_before();
     __syncwarp();
     cluster_sync();  // no DSMEM traffic may target a CTA that has exited
     tc_fence_after();
     if (warp == AT_MMA_WARP) tmem_dealloc(tmem, 512);
+}
+
+// CTA pairs of this shape that can be resident at once (the persistent grid).
+template <int NST, bool VSEP, int NPB, int NSX>
+static int attn_pairs_resident() {
+    static int cached = 0;
+    if (cached > 0) return cached;
+    using Lay = AtLayout<NST, VSEP, NPB, NSX>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 1024, 1, 1);
+    cfg.blockDim = dim3(AT_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Lay::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)attn_tc_kernel<NST, VSEP, NPB, NSX>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    if (n > 0) cached = n;
+    return n;
 }
 
 template <int NST, bool VSEP, int NPB, int NSX>
@@ -545,7 +714,10 @@ static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
     if (cudaFuncSetAttribute(attn_tc_kernel<NST, VSEP, NPB, NSX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Lay::SMEM) != cudaSuccess)
         return false;
-    attn_tc_kernel<NST, VSEP, NPB, NSX><<<(unsigned)(2 * a.total_q), AT_THREADS, Lay::SMEM, s>>>(a);
+    const int pairs = attn_pairs_resident<NST, VSEP, NPB, NSX>();
+    if (pairs <= 0) return false;
+    const int64_t grid_pairs = a.total_q < pairs ? a.total_q : pairs;
+    attn_tc_kernel<NST, VSEP, NPB, NSX><<<(unsigned)(2 * grid_pairs), AT_THREADS, Lay::SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }
 
@@ -557,7 +729,7 @@ static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
 
 bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s) {
     if (a.total_q <= 0) return true;
-    return a.v_separate ? launch_attn_tc_t<2, true, 2, 2>(a, s)
+    return a.v_separate ? launch_attn_tc_t<2, true, 2, 1>(a, s)
                         : launch_attn_tc_t<DSA_ATTN_NST, false, DSA_ATTN_NPB, DSA_ATTN_NSX>(a, s);
 }
 
