@@ -97,14 +97,18 @@ struct AtLayout {
     static constexpr uint32_t OFF_VM = OFF_LXR + 512;             // [2][64] validity bits of 2048 slots
     static constexpr uint32_t OFF_INFO = OFF_VM + 512;            // [2][8] last used slot per producer warp, [8] tile counts
     static constexpr uint32_t OFF_BAR = OFF_INFO + 128;
-    static constexpr uint32_t SMEM = OFF_BAR + 512;
+    // epilogue staging: per softmax warp 32 rows x 64 output columns (bf16),
+    // so that the output stores cover whole 128-byte lines
+    static constexpr bool EPI_STAGE = !VSEP;
+    static constexpr uint32_t OFF_EPI = OFF_BAR + 512;
+    static constexpr uint32_t SMEM = OFF_EPI + (EPI_STAGE ? 8 * 4096 : 0);
 };
 
 struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
     uint64_t s_full[2], s_empty[2];
-    uint64_t q_full;         // Q of the next query with tiles is in place (8 softmax warps)
+    uint64_t q_full;         // Q of the next query with tiles is in place (4 A warps)
     uint64_t o_full;         // all PVs of a query done
     uint64_t o_free;         // its epilogue has read O (8 softmax warps)
     uint64_t p_full[2];      // 4 local B warps + the peer's half of P (bytes)
@@ -166,7 +170,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             mbar_init(smem_u32(&bars->info_full[i]), AT_PRODUCERS);
             mbar_init(smem_u32(&bars->info_empty[i]), 9);
         }
-        mbar_init(smem_u32(&bars->q_full), 8);
+        mbar_init(smem_u32(&bars->q_full), 4);
         mbar_init(smem_u32(&bars->o_full), 1);
         mbar_init(smem_u32(&bars->o_free), 8);
         mbar_init(smem_u32(&bars->lx_full), 1);
@@ -237,6 +241,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
             for (int w = 0; w < AT_PRODUCERS; ++w) mx = max(mx, pmax[slot * 8 + w]);
             const int n_tiles = (mx + AT_N) / AT_N;
+            // ---- pull the next query's index row and Q rows into L2 while this
+            // query's tiles run (its scan and Q load then hit L2) ----
+            if (qi + 1 < nq) {
+                const int64_t tn = t + npairs;
+                if (warp == 0) {
+                    const char* ir = (const char*)(a.idx + tn * a.ld_idx);
+                    for (int off = (int)lane * 128; off < a.k_sel * 4; off += 32 * 128) prefetch_l2(ir + off);
+                } else if (warp <= 4) {
+                    const int hh = (int)(warp - 1) * 32 + (int)lane;
+                    const char* qr = (const char*)(a.q + tn * a.q_stride_tok + (int64_t)hh * a.q_stride_head + col0);
+                    for (int kb = 0; kb < nb; ++kb) prefetch_l2(qr + kb * 128);
+                }
+            }
             // ---- the query's tiles ----
             int32_t nxt[3] = {-1, -1, -1};
             auto load_idx = [&](int j) {
@@ -452,7 +469,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             tc_fence_after();
             const bool have_o = l_tot > 0.f;
             const float inv = have_o ? 1.0f / l_tot : 0.f;
-            __nv_bfloat16* orow = a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol;
             uint32_t r[4][32];
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + TM_O + ocol + c * 32, r[c]);
@@ -460,18 +476,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->o_free));  // O may be overwritten now
+            uint4 w[16];  // this row's 128 output columns, bf16
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint4* dst = (uint4*)(orow + c * 32);
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    uint4 w;
-                    w.x = pack_bf16(__uint_as_float(r[c][8 * i + 0]) * inv, __uint_as_float(r[c][8 * i + 1]) * inv);
-                    w.y = pack_bf16(__uint_as_float(r[c][8 * i + 2]) * inv, __uint_as_float(r[c][8 * i + 3]) * inv);
-                    w.z = pack_bf16(__uint_as_float(r[c][8 * i + 4]) * inv, __uint_as_float(r[c][8 * i + 5]) * inv);
-                    w.w = pack_bf16(__uint_as_float(r[c][8 * i + 6]) * inv, __uint_as_float(r[c][8 * i + 7]) * inv);
-                    dst[i] = w;
+                    w[4 * c + i].x = pack_bf16(__uint_as_float(r[c][8 * i + 0]) * inv, __uint_as_float(r[c][8 * i + 1]) * inv);
+                    w[4 * c + i].y = pack_bf16(__uint_as_float(r[c][8 * i + 2]) * inv, __uint_as_float(r[c][8 * i + 3]) * inv);
+                    w[4 * c + i].z = pack_bf16(__uint_as_float(r[c][8 * i + 4]) * inv, __uint_as_float(r[c][8 * i + 5]) * inv);
+                    w[4 * c + i].w = pack_bf16(__uint_as_float(r[c][8 * i + 6]) * inv, __uint_as_float(r[c][8 * i + 7]) * inv);
                 }
+            if constexpr (Lay::EPI_STAGE) {
+                // through this warp's staging tile: row = lane, 16-byte chunk k of a
+                // 64-column half at ((k ^ (row & 7)) << 4); read back as 4 rows x
+                // 128 bytes per instruction
+                uint8_t* stg = smem + Lay::OFF_EPI + (warp - AT_SOFT0) * 4096;
+                __nv_bfloat16* obase = a.out + t * a.out_stride_tok + (int64_t)(quad * 32) * a.out_stride_head + dv0 + ocol;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) *(uint4*)(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) = w[8 * half + k];
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = 4 * i + (int)(lane >> 3), k = (int)(lane & 7);
+                        const uint4 v = *(const uint4*)(stg + row * 128 + ((k ^ (row & 7)) << 4));
+                        *(uint4*)(obase + (int64_t)row * a.out_stride_head + half * 64 + k * 8) = v;
+                    }
+                    __syncwarp();
+                }
+            } else {
+                uint4* dst = (uint4*)(a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dst[i] = w[i];
             }
             if (rank == 0 && is_b && a.lse)
                 a.lse[t * 128 + h] = have_o ? (m_used + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
@@ -504,31 +541,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 if (rank == 0 && is_b && a.lse) a.lse[t * 128 + h] = -INFINITY;
                 continue;
             }
-            // ---- Q of this query -> TMEM (A operand of S = Q K^T); every S of the
-            // earlier queries has completed (this warp saw its s_full) ----
-            {
+            // ---- Q of this query -> TMEM (A operand of S = Q K^T), by the A warps,
+            // which finish a query's tiles first; every S of the earlier queries
+            // has completed (this warp saw its s_full) ----
+            if (!is_b) {
                 const __nv_bfloat16* qrow = a.q + t * a.q_stride_tok + (int64_t)h * a.q_stride_head + col0;
-                uint4 qreg[3][8];
+                uint4 qreg[5][8];
 #pragma unroll
-                for (int i = 0; i < 3; ++i) {
-                    const int kb = 2 * i + (is_b ? 1 : 0);
+                for (int kb = 0; kb < 5; ++kb) {
                     if (kb < nb) {
                         const uint4* src = (const uint4*)(qrow + kb * 64);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) qreg[i][j] = __ldg(src + j);
+                        for (int j = 0; j < 8; ++j) qreg[kb][j] = __ldg(src + j);
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 3; ++i) {
-                    const int kb = 2 * i + (is_b ? 1 : 0);
+                for (int kb = 0; kb < 5; ++kb) {
                     if (kb >= nb) continue;
                     uint32_t r[32];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        r[4 * j] = qreg[i][j].x;
-                        r[4 * j + 1] = qreg[i][j].y;
-                        r[4 * j + 2] = qreg[i][j].z;
-                        r[4 * j + 3] = qreg[i][j].w;
+                        r[4 * j] = qreg[kb][j].x;
+                        r[4 * j + 1] = qreg[kb][j].y;
+                        r[4 * j + 2] = qreg[kb][j].z;
+                        r[4 * j + 3] = qreg[kb][j].w;
                     }
                     if (kb < 4) {
                         tmem_st32(tmem + lane_off + TM_Q + kb * 32, r);

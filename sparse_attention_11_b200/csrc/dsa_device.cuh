@@ -206,6 +206,8 @@ DSA_DEV void st_async_b32(uint32_t addr, uint32_t a, uint32_t remote_bar) {
                  "r"(remote_bar)
                  : "memory");
 }
+// Hint: bring the 128-byte line holding p into L2.
+DSA_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"((uint64_t)p)); }
 DSA_DEV void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
