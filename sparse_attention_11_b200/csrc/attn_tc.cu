@@ -39,25 +39,29 @@
 // Pipelining.  Stage A (read S, send the partial) and stage B (combine,
 // probabilities, write P) run in separate warps, so consecutive tiles overlap;
 // the MMA warp issues greedily from two cursors: PV(u) as soon as P(u) is
-// complete, else S(t) as soon as its K/V stage is full and the S buffer is
-// free.  P tiles are double-buffered and released by a tcgen05.commit that
+// complete, else S(t) as soon as its K/V stage is full and the S accumulators
+// are free.  A tcgen05.mma takes about 50 cycles to issue from one thread,
+// which makes the 16-20 N=64 MMAs of an S tile issue-bound; so two warps issue
+// an S tile, each half of the contraction blocks into its own accumulator, and
+// the softmax warps add the two.  P tiles are double-buffered and released by a tcgen05.commit that
 // arrives on the p_free barrier of both CTAs (PV(t) done in both), so stage B
 // waits for PV(t-2), and for PV(t-1) only when the running maximum moves.
 // The P exchange also keeps the two CTAs within one tile of each other, which
 // the two-arrival p_free barrier relies on.
 //
-// Gathers: seven producer warps copy the selected rows with 16-byte
+// Gathers: six producer warps copy the selected rows with 16-byte
 // cp.async, 4 rows x 128 bytes per warp instruction, into the
 // 128-byte-swizzled tile layout the MMA reads (row r's 16-byte chunk c at
 // chunk c ^ (r & 7)).  Gather throughput grows with the number of issuing
 // warps, so the producers are many and small (setmaxnreg moves their
 // registers to the softmax warps).
 //
-// Tensor memory per CTA: O [0,256)  S [256,384) (two buffers)  Q [384,512)
-// (four 64-column blocks; rank 1's fifth block, the rope part, is read from
-// shared memory by SS MMAs).
-// Warps: 0-6 producers, 7 MMA issuer (+TMEM owner), 8-15 softmax / exchange /
-// epilogue: an A and a B warp per TMEM lane quadrant (thread <-> head).
+// Tensor memory per CTA: O [0,256)  S [256,384) (two partial accumulators)
+// Q [384,512) (four 64-column blocks; rank 1's fifth block, the rope part, is
+// read from shared memory by SS MMAs).
+// Warps: 0-5 producers, 6 second S issuer, 7 MMA issuer (+TMEM owner), 8-15
+// softmax / exchange / epilogue: an A and a B warp per TMEM lane quadrant
+// (thread <-> head).
 #include "dsa_kernels.h"
 
 namespace dsa {
@@ -69,6 +73,9 @@ namespace dsa {
 // pieces; for P it is also the no-swizzle K-major operand layout of the MMA
 // (8-row x 16-byte core matrices, 128 B apart along M and 2048 B along K).
 __device__ __forceinline__ uint32_t chunk_off(int h, int c) { return (uint32_t)(c * 2048 + h * 16); }
+#ifndef DSA_ATTN_EPI_STAGE
+#define DSA_ATTN_EPI_STAGE 1
+#endif
 constexpr int AT_N = 64;                           // keys per tile
 constexpr uint32_t AT_BLK = AT_N * 128;            // one 64-column block of a tile
 constexpr uint32_t AT_KST = 5 * AT_BLK;            // K part of a stage (max 5 blocks)
@@ -77,9 +84,10 @@ constexpr uint32_t AT_TILE128 = 128 * 128;         // a 128-row x 128-byte tile
 constexpr uint32_t AT_SX_BYTES = 128 * 128 + 128 * 4;  // partial scores + partial maxima
 constexpr uint32_t AT_PX_BYTES = 128 * 64;         // the peer's half of P
 constexpr uint32_t AT_LX_BYTES = 128 * 4;          // the peer's row sums
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;  // S: two 64-column buffers
-constexpr int AT_THREADS = 512;  // 7 producer + 1 MMA + 8 softmax warps
-constexpr int AT_PRODUCERS = 7;
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;  // S: two 64-column partial accumulators
+constexpr int AT_THREADS = 512;  // 6 producer + 2 MMA + 8 softmax warps
+constexpr int AT_PRODUCERS = 6;
+constexpr int AT_MMA2_WARP = 6;  // issues the second half of every S tile
 constexpr int AT_MMA_WARP = 7;
 constexpr int AT_SOFT0 = 8;      // first softmax warp (a warpgroup boundary)
 constexpr int AT_SCAN_ROUNDS = (2048 / 32 + AT_PRODUCERS - 1) / AT_PRODUCERS;  // index-row words per producer warp
@@ -99,7 +107,7 @@ struct AtLayout {
     static constexpr uint32_t OFF_BAR = OFF_INFO + 128;
     // epilogue staging: per softmax warp 32 rows x 64 output columns (bf16),
     // so that the output stores cover whole 128-byte lines
-    static constexpr bool EPI_STAGE = !VSEP;
+    static constexpr bool EPI_STAGE = !VSEP && DSA_ATTN_EPI_STAGE;
     static constexpr uint32_t OFF_EPI = OFF_BAR + 512;
     static constexpr uint32_t SMEM = OFF_EPI + (EPI_STAGE ? 8 * 4096 : 0);
 };
@@ -107,7 +115,8 @@ struct AtLayout {
 struct AtBars {
     uint64_t full[4];
     uint64_t empty[4];
-    uint64_t s_full[2], s_empty[2];
+    uint64_t s_full, s_empty;  // the S tile (both issuers committed) / read by the 8 softmax warps
+    uint64_t s_go;             // the second issuer may issue its half of the next S tile
     uint64_t q_full;         // Q of the next query with tiles is in place (4 A warps)
     uint64_t o_full;         // all PVs of a query done
     uint64_t o_free;         // its epilogue has read O (8 softmax warps)
@@ -120,6 +129,8 @@ struct AtBars {
     uint64_t drain;
     uint64_t info_full[2];   // query info published (7 producer warps)
     uint64_t info_empty[2];  // query info consumed (MMA warp + 8 softmax warps)
+    uint64_t drain2;
+    int go[2];  // stage of the S tile announced on s_go, -1: no more tiles
     uint32_t tmem_base;
     int abort;
 };
@@ -160,9 +171,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             mbar_init(smem_u32(&bars->full[i]), AT_PRODUCERS * 32);
             mbar_init(smem_u32(&bars->empty[i]), 1);
         }
+        mbar_init(smem_u32(&bars->s_full), 2);   // one commit per issuer
+        mbar_init(smem_u32(&bars->s_empty), 8);  // 4 A + 4 B warps read every S tile
+        mbar_init(smem_u32(&bars->s_go), 1);
+        mbar_init(smem_u32(&bars->drain2), 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&bars->s_full[i]), 1);
-            mbar_init(smem_u32(&bars->s_empty[i]), 8);  // 4 A + 4 B warps read every S tile
             mbar_init(smem_u32(&bars->p_full[i]), 4);   // (only NPB of them are used)
             mbar_init(smem_u32(&bars->p_free[i]), 2);
             mbar_init(smem_u32(&bars->sx_full[i]), 1);
@@ -193,6 +206,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     const uint32_t s_stage0 = smem_u32(smem);
     const uint32_t s_p0 = smem_u32(smem + Lay::OFF_P);
     const uint32_t s_qr = smem_u32(smem + Lay::OFF_QR);
+    // Half hf of the S tile of stage s: K-blocks 2hf, 2hf+1 (Q from TMEM) and, on
+    // rank 1, K-steps 2hf, 2hf+1 of the rope block (Q from shared memory), into
+    // accumulator hf.  Issued by one thread.
+    auto s_half = [&](int hf, uint32_t s) {
+        constexpr uint32_t idesc_s = idesc_make(1, 1, false, 128, AT_N);
+        const uint32_t kst = s_stage0 + s * Lay::STAGE;
+        const uint32_t d = tmem + TM_S + 64 * hf;
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+            const int kb = 2 * hf + k2;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ts(d, tmem + TM_Q + kb * 32 + ks * 8, sdesc_sw128(kst + kb * AT_BLK + ks * 32, 16, 1024), idesc_s,
+                            (k2 | ks) ? 1u : 0u);
+        }
+        if (nb == 5)
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const int ks = 2 * hf + k2;
+                mma_bf16_ss(d, sdesc_sw128(s_qr + ks * 32, 16, 1024), sdesc_sw128(kst + 4 * AT_BLK + ks * 32, 16, 1024),
+                            idesc_s, 1u);
+            }
+    };
     if (warp < AT_PRODUCERS) {
         // ================= gather producers (7 warps) =================
         asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
@@ -298,7 +334,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     } else if (warp == AT_MMA_WARP) {
         // ================= MMA issuer =================
         asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
-        constexpr uint32_t idesc_s = idesc_make(1, 1, false, 128, AT_N);
         constexpr uint32_t idesc_pv = idesc_make(1, 1, true, 128, 256);
         // Two cursors over the pair's tile sequence.  S cursor: query qs (ns
         // tiles once its info is read, else -1), tile js, sequence tile gs,
@@ -361,28 +396,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                         done = true;
                     }
                 } else {
-                    const uint32_t s = gs % NST, sb = gs & 1;
+                    const uint32_t s = gs % NST;
                     bool rdy = mbar_probe(smem_u32(&bars->full[s]), (gs / NST) & 1) &&
-                               mbar_probe(smem_u32(&bars->s_empty[sb]), ((gs >> 1) & 1) ^ 1);
+                               mbar_probe(smem_u32(&bars->s_empty), (gs & 1) ^ 1);
                     if (js == 0) rdy = rdy && mbar_probe(smem_u32(&bars->q_full), nqs & 1);
                     if (__all_sync(0xffffffffu, rdy)) {
                         fence_proxy_async();
                         tc_fence_after();
                         if (lane == 0) {
-                            const uint32_t kst = s_stage0 + s * Lay::STAGE;
-                            const uint32_t d = tmem + TM_S + 64 * sb;
-                            for (int kb = 0; kb < 4; ++kb)
-#pragma unroll
-                                for (int ks = 0; ks < 4; ++ks)
-                                    mma_bf16_ts(d, tmem + TM_Q + kb * 32 + ks * 8,
-                                                sdesc_sw128(kst + kb * AT_BLK + ks * 32, 16, 1024), idesc_s,
-                                                (kb | ks) ? 1u : 0u);
-                            if (nb == 5)  // the rope block: Q from shared memory
-#pragma unroll
-                                for (int ks = 0; ks < 4; ++ks)
-                                    mma_bf16_ss(d, sdesc_sw128(s_qr + ks * 32, 16, 1024),
-                                                sdesc_sw128(kst + 4 * AT_BLK + ks * 32, 16, 1024), idesc_s, 1u);
-                            mma_commit(smem_u32(&bars->s_full[sb]));
+                            // first half of S: blocks 0, 1 (+ rope K-steps 0, 1); the
+                            // second issuer adds blocks 2, 3 (+ rope 2, 3) into its own
+                            // accumulator
+                            bars->go[gs & 1] = (int)s;
+                            mbar_arrive(smem_u32(&bars->s_go));
+                            s_half(0, s);
+                            mma_commit(smem_u32(&bars->s_full));
                         }
                         __syncwarp();
                         ++gs;
@@ -412,9 +440,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 }
             }
         }
+        if (ok && lane == 0) {  // no more S tiles
+            bars->go[gs & 1] = -1;
+            mbar_arrive(smem_u32(&bars->s_go));
+        }
         if (*abort && lane == 0) {
             mma_commit(smem_u32(&bars->drain));
             mbar_wait(smem_u32(&bars->drain), 0, nullptr, st, 0x2205, 1ll << 28);
+        }
+    } else if (warp == AT_MMA2_WARP) {
+        // ================= second S issuer =================
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        for (uint32_t g = 0;; ++g) {
+            if (!wait_warp(smem_u32(&bars->s_go), g & 1, abort, st, 0x2401)) break;
+            const int s = *(volatile int*)&bars->go[g & 1];
+            if (s < 0) break;
+            fence_proxy_async();
+            tc_fence_after();
+            if (lane == 0) {
+                s_half(1, (uint32_t)s);
+                mma_commit(smem_u32(&bars->s_full));
+            }
+            __syncwarp();
+        }
+        if (*abort && lane == 0) {
+            mma_commit(smem_u32(&bars->drain2));
+            mbar_wait(smem_u32(&bars->drain2), 0, nullptr, st, 0x2405, 1ll << 28);
         }
     } else {
         // ================= softmax / exchange / epilogue (8 warps) =================
@@ -591,41 +642,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             }
             float m_used = -INFINITY, l = 0.f;
             for (int u = 0; ok && u < n_tiles; ++u, ++g) {
-                const uint32_t b = g & 1, ph = (g >> 1) & 1;          // S buffer and its phase
                 const uint32_t xb = g % NSX, xph = (g / NSX) & 1;      // partial-score buffer and its phase
                 const uint32_t mlo = vmask[slot * 64 + 2 * u], mhi = vmask[slot * 64 + 2 * u + 1];
-                if (!wait_warp(smem_u32(&bars->s_full[b]), ph, abort, st, 0x2301)) { ok = false; break; }
+                if (!wait_warp(smem_u32(&bars->s_full), g & 1, abort, st, 0x2301)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_off + TM_S + 64 * b, r0);
-                tmem_ld32(tmem + lane_off + TM_S + 64 * b + 32, r1);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[b]));
-                float pm = -INFINITY;  // partial maximum of this CTA's row over the tile's valid keys
+                // this CTA's partial S = accumulator 0 + accumulator 1; the peer's key
+                // half first (stage A sends it on), then this CTA's own half
+                const uint32_t ta = tmem + lane_off + TM_S;
+                const int ph_ = kh ^ 1, oh = kh;  // key halves: the peer's, this CTA's
+                uint32_t rp[32], ro[32];
+                {
+                    uint32_t x[32];
+                    tmem_ld32(ta + 32 * ph_, rp);
+                    tmem_ld32(ta + 64 + 32 * ph_, x);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    if ((mlo >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r0[i]));
-                    if ((mhi >> i) & 1u) pm = fmaxf(pm, __uint_as_float(r1[i]));
+                    for (int i = 0; i < 32; ++i) rp[i] = __float_as_uint(__uint_as_float(rp[i]) + __uint_as_float(x[i]));
                 }
                 if (!is_b) {
-                    // ---- stage A: send the peer's 32 partial columns and the partial max ----
+                    // ---- stage A: send the peer's 32 partial columns, then the partial max ----
                     if (!wait_warp(my_sx_free0 + 8 * xb, xph ^ 1, abort, st, 0x2302)) { ok = false; break; }
                     const uint32_t dst = peer_sx + xb * AT_TILE128;
                     const uint32_t bar = peer_sx_full0 + 8 * xb;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {  // the peer's keys: [32,64) for rank 0, [0,32) for rank 1
-                        uint32_t w[4];
+                    for (int c = 0; c < 8; ++c)
+                        st_async_v4(dst + chunk_off(h, c), rp[4 * c], rp[4 * c + 1], rp[4 * c + 2], rp[4 * c + 3], bar);
+                }
+                {
+                    uint32_t x[32];
+                    tmem_ld32(ta + 32 * oh, ro);
+                    tmem_ld32(ta + 64 + 32 * oh, x);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) w[e] = kh ? r0[4 * c + e] : r1[4 * c + e];
-                        st_async_v4(dst + chunk_off(h, c), w[0], w[1], w[2], w[3], bar);
-                    }
-                    st_async_b32(peer_pm + xb * 512 + h * 4, __float_as_uint(pm), bar);
+                    for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) + __uint_as_float(x[i]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
+                const uint32_t mo = kh ? mhi : mlo, mp = kh ? mlo : mhi;  // valid slots of the own / peer half
+                float pm = -INFINITY;  // partial maximum of this CTA's row over the tile's valid keys
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if ((mo >> i) & 1u) pm = fmaxf(pm, __uint_as_float(ro[i]));
+                    if ((mp >> i) & 1u) pm = fmaxf(pm, __uint_as_float(rp[i]));
+                }
+                if (!is_b) {
+                    st_async_b32(peer_pm + xb * 512 + h * 4, __float_as_uint(pm), peer_sx_full0 + 8 * xb);
                     continue;
                 }
                 // ---- stage B: combine, probabilities, both copies of P ----
-                const uint32_t msk = kh ? mhi : mlo;
+                const uint32_t msk = mo;
                 if (!wait_warp(my_sx_full0 + 8 * xb, xph, abort, st, 0x2303)) { ok = false; break; }
                 if (arm_thread) mbar_arrive_expect_tx(my_sx_full0 + 8 * xb, AT_SX_BYTES);  // its next phase
                 float s32[32];
@@ -637,7 +703,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                         const float pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            s32[4 * c + e] = __uint_as_float(kh ? r1[4 * c + e] : r0[4 * c + e]) + pv[e];
+                            s32[4 * c + e] = __uint_as_float(ro[4 * c + e]) + pv[e];
                     }
                 }
                 const float pm_peer = pmx[xb * 128 + h];
