@@ -9,14 +9,17 @@
 // L x L score matrix never leaves the SM).
 //
 // Work unit: a block of 128 consecutive queries of one sequence.  One CTA
-// per block, 6 warps:
+// per block, 10 warps:
 //   warp 0      TMA producer: the block's folded queries (128 x 128 e4m3,
 //               once) and key tiles of 256 x 128 e4m3 (+ their fp32 scales)
 //   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f8f6f4,
 //               M=128 N=256 K=32, fp32 accumulators in two TMEM buffers
-//   warps 2..5  epilogue: thread <-> query row (its TMEM lane); reads a
-//               row of 256 fp32 dots per tile, forms the score
-//               ReLU((dot * s_k) * s_row) and applies the sweep's action.
+//   warps 2..9  epilogue: two threads per query row (its TMEM lane), one per
+//               128-column half of each tile; each reads its 128 fp32 dots
+//               per tile, forms the score ReLU((dot * s_k) * s_row) and
+//               applies the sweep's action.  The two halves share the row's
+//               histogram (shared-memory atomics) and, when emitting, trade
+//               their per-tile counts so the indices stay in ascending order.
 //
 // Sweeps over the block's causal key tiles (a block stops as soon as every
 // row's selection is determined):
@@ -44,7 +47,10 @@ constexpr uint32_t IX_OFF_A = 0;
 constexpr uint32_t IX_OFF_B = IX_OFF_A + IX_A_BYTES;
 constexpr uint32_t IX_OFF_SC = IX_OFF_B + IX_NST * IX_B_BYTES;
 constexpr uint32_t IX_OFF_HIST = IX_OFF_SC + IX_NST * IX_BN * 4;
-constexpr uint32_t IX_OFF_BAR = IX_OFF_HIST + 256 * IX_BM * 4;
+constexpr uint32_t IX_OFF_ECNT = IX_OFF_HIST + 256 * IX_BM * 4;    // [2 tiles][2 halves][128 rows] uint2
+constexpr uint32_t IX_OFF_BAR = IX_OFF_ECNT + 2 * 2 * IX_BM * 8;
+constexpr int IX_EPI_WARPS = 8;
+constexpr int IX_THREADS = 64 + 32 * IX_EPI_WARPS;
 constexpr uint32_t IX_SMEM = IX_OFF_BAR + 256 + 1024;  // + alignment slack
 
 enum : int { SW_STOP = 0, SW_HIST = 1, SW_EMIT = 2, SW_SCORES = 3 };
@@ -150,13 +156,14 @@ __device__ __forceinline__ void ep_chunk(uint32_t (&v)[32], const float* scs, fl
 }
 #undef KB
 
-// All 256 columns of a tile for one row, one 32-column TMEM load at a time.
+// One 128-column half of a tile for one row (taddr, scs and s_tile already
+// point at the half), one 32-column TMEM load at a time.
 template <int MODE>
 __device__ __forceinline__ void ep_tile(uint32_t taddr, bool ok, bool active, const float* scs, float srow, int64_t pos,
                                         int64_t s_tile, RowSel& rs, uint32_t* myhist, int dshift, uint32_t dmask,
                                         int32_t* out, int kcap, float* srow_out) {
 #pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
+    for (int ch = 0; ch < 4; ++ch) {
         uint32_t v[32];
         if (ok) {
             tmem_ld32(taddr + ch * 32, v);
@@ -170,7 +177,76 @@ __device__ __forceinline__ void ep_tile(uint32_t taddr, bool ok, bool active, co
     }
 }
 
-__global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constant__ IndexerTcArgs a) {
+// EMIT for one 128-column half of a tile.  Both halves of the row form their
+// masks, trade (above, equal) counts through shared memory (slot ec, this
+// half's counts at ec[half], the partner's at ec[half ^ 1]) with a two-warp
+// barrier, then write their keys at their places in the ascending order: the
+// first half's keys precede the second half's, the bucket's equal keys are
+// taken in index order until the row has what it needs.
+__device__ __forceinline__ void ep_emit_half(uint32_t taddr, bool ok, bool active, const float* scs, float srow, int64_t pos,
+                                             int64_t s_half, int half, RowSel& rs, int32_t* out, int kcap, uint2* ec,
+                                             int bar_id) {
+    // ec[h * IX_BM]: the counts of half h of this row
+    uint32_t abv[4], eqm[4];
+    uint32_t n_above = 0, n_eq = 0;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t v[32];
+        if (ok) {
+            tmem_ld32(taddr + ch * 32, v);
+            tmem_wait_ld();
+        }
+        abv[ch] = 0;
+        eqm[ch] = 0;
+        const int64_t sb = s_half + ch * 32;
+        if (!active || sb > pos) continue;
+        chunk_keys(v, scs + ch * 32, srow);
+        const int lim = (int)min((int64_t)31, pos - sb);
+        const uint32_t limmask = lim >= 31 ? 0xFFFFFFFFu : ((1u << (lim + 1)) - 1u);
+        uint32_t above = 0, eq = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int hi = ((int)v[i] - 1) >> rs.sh;
+            above |= (uint32_t)(hi > rs.P) << i;
+            eq |= (uint32_t)(hi == rs.P) << i;
+        }
+        if (rs.take_all) above = 0xFFFFFFFFu, eq = 0;
+        abv[ch] = above & limmask;
+        eqm[ch] = eq & limmask;
+        n_above += __popc(abv[ch]);
+        n_eq += __popc(eqm[ch]);
+    }
+    ec[half * IX_BM] = make_uint2(n_above, n_eq);
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+    const uint2 c0 = half ? ec[0] : make_uint2(n_above, n_eq);
+    const uint2 c1 = half ? make_uint2(n_above, n_eq) : ec[IX_BM];
+    const uint32_t left = rs.need > rs.taken ? rs.need - rs.taken : 0u;
+    const uint32_t t0 = min(c0.y, left), t1 = min(c1.y, left - t0);
+    int pos_out = rs.cnt + (half ? (int)(c0.x + t0) : 0);
+    uint32_t take = half ? t1 : t0;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t any = abv[ch] | eqm[ch];
+        const int32_t sb = (int32_t)(s_half + ch * 32);
+        while (any) {
+            const int i = __ffs(any) - 1;
+            any &= any - 1;
+            bool e = (abv[ch] >> i) & 1u;
+            if (!e && take > 0) {
+                e = true;
+                --take;
+            }
+            if (e) {
+                if (pos_out < kcap) out[pos_out] = sb + i;
+                ++pos_out;
+            }
+        }
+    }
+    rs.cnt += (int)(c0.x + t0 + c1.x + t1);
+    rs.taken += t0 + t1;
+}
+
+__global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_constant__ IndexerTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     IxBars* bars = (IxBars*)(smem + IX_OFF_BAR);
@@ -210,11 +286,11 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
     if (threadIdx.x == 0) {
         for (int i = 0; i < IX_NST; ++i) {
             mbar_init(smem_u32(&bars->full[i]), 1);
-            mbar_init(smem_u32(&bars->empty[i]), 1 + 4);
+            mbar_init(smem_u32(&bars->empty[i]), 1 + IX_EPI_WARPS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&bars->acc_full[i]), 1);
-            mbar_init(smem_u32(&bars->acc_empty[i]), 4);
+            mbar_init(smem_u32(&bars->acc_empty[i]), IX_EPI_WARPS);
         }
         mbar_init(smem_u32(&bars->a_full), 1);
         mbar_init(smem_u32(&bars->dec), 1);
@@ -312,8 +388,9 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
             }
         }
     } else {
-        // ================= epilogue: thread <-> query row =================
+        // ================= epilogue: two threads per query row =================
         const uint32_t quad = warp & 3;
+        const int half = (int)(warp - 2) >> 2;  // 128-column half of every tile
         const int row = (int)(quad * 32 + lane);
         const bool has_row = row < nrows;
         const int64_t t = t_first + row;
@@ -334,7 +411,8 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
         uint32_t* myhist = hist + row;  // bin b at myhist[b * IX_BM]
         int32_t* out = (a.mode == 0 && has_row) ? a.idx + t * a.ld_idx : nullptr;
         float* srow_out = (a.mode == 1 && has_row && in_range) ? a.scores + (t - a.row_begin) * a.ld_scores : nullptr;
-        for (int i = 0; i < 256; ++i) myhist[i * IX_BM] = 0;
+        for (int i = 128 * half; i < 128 * half + 128; ++i) myhist[i * IX_BM] = 0;
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // both halves cleared the row's bins
 
         uint32_t g = 0;
         int kind = first_kind;
@@ -345,17 +423,18 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
                 bool ok = wait_warp(smem_u32(&bars->acc_full[ab]), (g >> 1) & 1, abort, st, 0x1301);
                 ok = ok && wait_warp(smem_u32(&bars->full[s]), (g / IX_NST) & 1, abort, st, 0x1302);
                 tc_fence_after();
-                const float* scs = sc_s + s * IX_BN;
-                const int64_t s_tile = (int64_t)tile * IX_BN;
+                const float* scs = sc_s + s * IX_BN + 128 * half;
+                const int64_t s_tile = (int64_t)tile * IX_BN + 128 * half;
                 const bool active = ok && has_row && !(kind == SW_HIST && resolved);
-                const uint32_t taddr = tmem + ((quad * 32) << 16) + ab * IX_BN;
+                const uint32_t taddr = tmem + ((quad * 32) << 16) + ab * IX_BN + 128 * half;
                 if (kind == SW_HIST && lvl == 1)
                     ep_tile<1>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
                 else if (kind == SW_HIST)
                     ep_tile<4>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, lvl == 2 ? 15 : lvl == 3 ? 7 : 0,
                                lvl == 4 ? 127u : 255u, out, a.k, srow_out);
                 else if (kind == SW_EMIT)
-                    ep_tile<2>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
+                    ep_emit_half(taddr, ok, active, scs, srow, pos, s_tile, half, rs, out, a.k,
+                                 (uint2*)(smem + IX_OFF_ECNT) + (tile & 1) * 2 * IX_BM + row, 2 + (int)quad);
                 else
                     ep_tile<3>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
                 tc_fence_before();
@@ -365,8 +444,11 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
                     mbar_arrive(smem_u32(&bars->empty[s]));
                 }
             }
-            // ---- end of sweep: refine each row's bucket; one thread decides ----
+            // ---- end of sweep: refine each row's bucket (both halves of the row
+            // reach the same decision from the shared histogram); one thread
+            // decides the next sweep ----
             if (kind == SW_HIST) {
+                asm volatile("bar.sync 1, 256;" ::: "memory");  // every count of the sweep is in
                 if (has_row && !resolved) {
                     uint32_t cum = 0;
                     int bsel = 0;
@@ -385,23 +467,23 @@ __global__ void __launch_bounds__(192, 1) indexer_tc_kernel(const __grid_constan
                     resolved = in_bin == rs.need || rs.P == -1 || lvl == 4;
                 }
                 level = lvl;
-                for (int i = 0; i < 256; ++i) myhist[i * IX_BM] = 0;
                 if (threadIdx.x == 64) bars->any_unresolved = 0;
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync 1, 256;" ::: "memory");  // every histogram read is done
+                for (int i = 128 * half; i < 128 * half + 128; ++i) myhist[i * IX_BM] = 0;
                 if (has_row && !resolved) bars->any_unresolved = 1;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             if (threadIdx.x == 64) {
                 int nk = kind == SW_HIST ? (bars->any_unresolved ? SW_HIST : SW_EMIT) : SW_STOP;
                 if (*abort) nk = SW_STOP;
                 bars->next_kind = nk;
                 mbar_arrive(smem_u32(&bars->dec));
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             kind = *(volatile int*)&bars->next_kind;
         }
         // ---- finish the index rows ----
-        if (a.mode == 0 && has_row) {
+        if (a.mode == 0 && has_row && half == 0) {
             if (first_kind == SW_STOP) {  // every row of the block keeps its whole prefix
                 for (int64_t s = 0; s <= pos; ++s) out[s] = (int32_t)s;
                 rs.cnt = (int)(pos + 1);
@@ -423,7 +505,7 @@ bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s) {
     const int64_t nblk = (a.max_seqlen_q + IX_BM - 1) / IX_BM;
     const int64_t grid = nblk * a.sv.batch;
     if (grid <= 0) return true;
-    indexer_tc_kernel<<<(unsigned)grid, 192, IX_SMEM, s>>>(a);
+    indexer_tc_kernel<<<(unsigned)grid, IX_THREADS, IX_SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }
 
