@@ -90,6 +90,18 @@ constexpr int AT_PRODUCERS = 6;
 constexpr int AT_MMA2_WARP = 6;  // issues the second half of every S tile
 constexpr int AT_MMA_WARP = 7;
 constexpr int AT_SOFT0 = 8;      // first softmax warp (a warpgroup boundary)
+// Register split (setmaxnreg): warpgroup 0 (producers 0-3) and warpgroup 1
+// (producers 4-5 and the two MMA warps) give registers to the softmax
+// warpgroups.  setmaxnreg.inc draws only on the registers the block was
+// launched with, so the split must fit the launch total (threads x registers
+// per thread at launch), or the softmax warps wait forever; the launcher
+// checks the compiled count before every launch.
+constexpr int AT_REGS_WG0 = 40;
+constexpr int AT_REGS_WG1 = 56;
+constexpr int AT_REGS_SOFT = 208;
+constexpr int AT_REGS_SPLIT = 128 * AT_REGS_WG0 + 128 * AT_REGS_WG1 + (AT_THREADS - 256) * AT_REGS_SOFT;
+static_assert(AT_SOFT0 == 8, "the register split assumes two producer/MMA warpgroups");
+static_assert(AT_REGS_SPLIT <= ((65536 / AT_THREADS) & ~7) * AT_THREADS, "register split above the launch total");
 constexpr int AT_SCAN_ROUNDS = (2048 / 32 + AT_PRODUCERS - 1) / AT_PRODUCERS;  // index-row words per producer warp
 constexpr int AT_NTAB = 8;       // tile counts of the queries between the PV and the S cursor
 
@@ -230,8 +242,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             }
     };
     if (warp < AT_PRODUCERS) {
-        // ================= gather producers (7 warps) =================
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        // ================= gather producers (6 warps) =================
+        if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(AT_REGS_WG0));
+        else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(AT_REGS_WG1));
         // 16 groups of 4 keys per tile; warp w takes groups w, w+7, w+14
         const int sub = (int)(lane >> 3), chunk = (int)(lane & 7);
         const int ngrp = (16 - (int)warp + AT_PRODUCERS - 1) / AT_PRODUCERS;
@@ -333,7 +346,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == AT_MMA_WARP) {
         // ================= MMA issuer =================
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(AT_REGS_WG1));
         constexpr uint32_t idesc_pv = idesc_make(1, 1, true, 128, 256);
         // Two cursors over the pair's tile sequence.  S cursor: query qs (ns
         // tiles once its info is read, else -1), tile js, sequence tile gs,
@@ -450,7 +463,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         }
     } else if (warp == AT_MMA2_WARP) {
         // ================= second S issuer =================
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(AT_REGS_WG1));
         for (uint32_t g = 0;; ++g) {
             if (!wait_warp(smem_u32(&bars->s_go), g & 1, abort, st, 0x2401)) break;
             const int s = *(volatile int*)&bars->go[g & 1];
@@ -476,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         // probabilities and write P.  Both groups run every tile concurrently.
         // Per query: load Q (after the previous query's last S), finish the
         // previous query (row sums, O / l), then the tiles.
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(AT_REGS_SOFT));
         const uint32_t quad = warp & 3;
         const bool is_b = warp >= AT_SOFT0 + 4;
         const int h = (int)(quad * 32 + lane);
@@ -815,6 +828,11 @@ static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
     static_assert(Lay::SMEM <= 232448, "shared memory budget");
     if (cudaFuncSetAttribute(attn_tc_kernel<NST, VSEP, NPB, NSX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Lay::SMEM) != cudaSuccess)
+        return false;
+    // the setmaxnreg split must fit the registers the block is launched with
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, (const void*)attn_tc_kernel<NST, VSEP, NPB, NSX>) != cudaSuccess ||
+        (int64_t)fa.numRegs * AT_THREADS < (int64_t)AT_REGS_SPLIT)
         return false;
     const int pairs = attn_pairs_resident<NST, VSEP, NPB, NSX>();
     if (pairs <= 0) return false;
