@@ -73,8 +73,12 @@ enum dsa_op {
     DSA_OP_INDEX_SCORES = 1,
     DSA_OP_TOPK = 2,
     DSA_OP_SPARSE_ATTN = 3,
-    DSA_OP_FORWARD = 4
+    DSA_OP_FORWARD = 4,
+    DSA_OP_FORWARD_HOST = 5
 };
+
+/* Query rows per chunk of dsa_forward_host. */
+#define DSA_HOST_CHUNK_ROWS 2048
 
 /* Packed variable-length batch (see "Sequences" above). */
 typedef struct dsa_seqs {
@@ -218,6 +222,30 @@ DSA_API int dsa_select_noalloc(const dsa_seqs* seqs, const dsa_indexer_args* ia,
 DSA_API int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa,
                 int32_t k, int32_t* idx_out, int64_t ld_idx, void* ws, size_t ws_bytes,
                 dsa_stream_t stream);
+
+/* dsa_forward with the attention query and output in HOST memory, for a
+ * caller whose activations live on the host.  aa->q and aa->out are host
+ * pointers (page-locked, e.g. cudaHostAlloc, so the copies run
+ * asynchronously); every other operand is a device pointer as in
+ * dsa_forward.  BF16 tensor-core attention only (heads 128, dk 576, dv 512),
+ * with packed q [total_q, 128, 576] and out [total_q, 128, 512]
+ * (q_stride_head = dk, q_stride_tok = heads*dk, likewise for out); other
+ * strides return DSA_ERR_INVALID_ARG.
+ *
+ * The selection (a1-a3) runs first on `stream` for all queries.  The
+ * attention then runs in chunks of DSA_HOST_CHUNK_ROWS query rows: chunk c's
+ * Q is copied in on `h2d_stream` while chunk c-1's attention runs on `stream`
+ * and chunk c-2's output is copied out on `d2h_stream`, so the two PCIe
+ * directions and the compute overlap.  Two device staging buffers each for Q
+ * and output chunks live in the workspace (DSA_OP_FORWARD_HOST).  The three
+ * streams may be the same stream (no overlap then).  The call returns once
+ * the work is enqueued; `stream` is ordered after the last output copy, so
+ * synchronising `stream` makes the host output visible.  Results are
+ * identical to dsa_forward's.  The paper has no counterpart: this is the
+ * host-memory front end of this library. */
+DSA_API int dsa_forward_host(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k,
+                             int32_t* idx_out, int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream,
+                             dsa_stream_t h2d_stream, dsa_stream_t d2h_stream);
 
 /* Synchronise `stream`, return the first device-side error recorded in the
  * workspace status header since the last call (DSA_OK if none), write its

@@ -93,6 +93,38 @@ WsLayout ws_layout(const dsa_seqs* s, const dsa_indexer_args* ia, int32_t k, boo
     return L;
 }
 
+// dsa_forward_host: the forward's workspace, then two device staging buffers
+// each for query and output chunks of DSA_HOST_CHUNK_ROWS rows.
+struct HostLayout {
+    WsLayout fwd;
+    size_t q[2], o[2], q_chunk_bytes, o_chunk_bytes, total;
+    int64_t chunk;
+};
+
+HostLayout host_layout(const dsa_seqs* s, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k) {
+    HostLayout H;
+    H.fwd = ws_layout(s, ia, k, true, !use_tc_indexer(s, ia));
+    H.chunk = s->total_q < DSA_HOST_CHUNK_ROWS ? s->total_q : DSA_HOST_CHUNK_ROWS;
+    H.q_chunk_bytes = (size_t)H.chunk * (size_t)aa->heads * (size_t)aa->dk * 2;
+    H.o_chunk_bytes = (size_t)H.chunk * (size_t)aa->heads * (size_t)aa->dv * 2;
+    size_t off = H.fwd.total;
+    for (int i = 0; i < 2; ++i) {
+        H.q[i] = off;
+        off = align256(off + H.q_chunk_bytes);
+    }
+    for (int i = 0; i < 2; ++i) {
+        H.o[i] = off;
+        off = align256(off + H.o_chunk_bytes);
+    }
+    H.total = off;
+    return H;
+}
+
+bool packed_q_out(const dsa_attn_args* aa) {
+    return aa->q_stride_head == aa->dk && aa->q_stride_tok == (int64_t)aa->heads * aa->dk &&
+           aa->out_stride_head == aa->dv && aa->out_stride_tok == (int64_t)aa->heads * aa->dv;
+}
+
 SeqView seq_view(const dsa_seqs* s) {
     SeqView v;
     v.batch = s->batch;
@@ -219,34 +251,41 @@ int run_topk(const dsa_seqs* s, const float* scores, int64_t ld, int64_t row_beg
     return cuda_status();
 }
 
+// Tensor-core attention over query rows [row_begin, row_begin + row_count);
+// q and out point at row row_begin.
+int run_attn_tc_rows(const dsa_seqs* s, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel,
+                     int64_t row_begin, int64_t row_count, const void* q, void* out, StatusHdr* h, cudaStream_t st) {
+    AttnTcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.sv = seq_view(s);
+    a.total_q = s->total_q;
+    a.q = (const __nv_bfloat16*)q;
+    a.q_stride_tok = aa->q_stride_tok;
+    a.q_stride_head = aa->q_stride_head;
+    a.scale_log2 = aa->scale * 1.4426950408889634f;
+    a.out = (__nv_bfloat16*)out;
+    a.out_stride_tok = aa->out_stride_tok;
+    a.out_stride_head = aa->out_stride_head;
+    a.lse = aa->lse;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.k_sel = k_sel;
+    a.v_separate = attn_v_separate(aa) ? 1 : 0;
+    a.st = h;
+    a.k = (const __nv_bfloat16*)aa->k;
+    a.k_stride = aa->k_stride;
+    a.v = (const __nv_bfloat16*)aa->v;
+    a.v_stride = aa->v_stride;
+    a.row_begin = row_begin;
+    a.row_count = row_count;
+    if (!launch_attn_tc(a, st)) return DSA_ERR_CUDA;
+    return cuda_status();
+}
+
 int run_attn(const dsa_seqs* s, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel, StatusHdr* h,
              cudaStream_t st) {
     if (s->total_q == 0) return DSA_OK;
-    if (attn_is_tc(aa)) {
-        AttnTcArgs a;
-        memset(&a, 0, sizeof(a));
-        a.sv = seq_view(s);
-        a.total_q = s->total_q;
-        a.q = (const __nv_bfloat16*)aa->q;
-        a.q_stride_tok = aa->q_stride_tok;
-        a.q_stride_head = aa->q_stride_head;
-        a.scale_log2 = aa->scale * 1.4426950408889634f;
-        a.out = (__nv_bfloat16*)aa->out;
-        a.out_stride_tok = aa->out_stride_tok;
-        a.out_stride_head = aa->out_stride_head;
-        a.lse = aa->lse;
-        a.idx = idx;
-        a.ld_idx = ld_idx;
-        a.k_sel = k_sel;
-        a.v_separate = attn_v_separate(aa) ? 1 : 0;
-        a.st = h;
-        a.k = (const __nv_bfloat16*)aa->k;
-        a.k_stride = aa->k_stride;
-        a.v = (const __nv_bfloat16*)aa->v;
-        a.v_stride = aa->v_stride;
-        if (!launch_attn_tc(a, st)) return DSA_ERR_CUDA;
-        return cuda_status();
-    }
+    if (attn_is_tc(aa)) return run_attn_tc_rows(s, aa, idx, ld_idx, k_sel, 0, s->total_q, aa->q, aa->out, h, st);
     AttnF32Launch L;
     L.sv = seq_view(s);
     L.a.heads = aa->heads;
@@ -294,7 +333,6 @@ int dsa_version(void) { return 1000; }
 
 int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexer_args* ia, const dsa_attn_args* aa,
                        size_t* bytes) {
-    (void)aa;
     if (!bytes) return DSA_ERR_INVALID_ARG;
     int r = check_seqs(seqs);
     if (r) return r;
@@ -309,6 +347,10 @@ int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexe
         case DSA_OP_FORWARD:
             if (!ia || k < 1) return DSA_ERR_INVALID_ARG;
             *bytes = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia)).total;
+            return DSA_OK;
+        case DSA_OP_FORWARD_HOST:
+            if (!ia || !aa || k < 1 || aa->heads < 1 || aa->dk < 1 || aa->dv < 1) return DSA_ERR_INVALID_ARG;
+            *bytes = host_layout(seqs, ia, aa, k).total;
             return DSA_OK;
     }
     return DSA_ERR_INVALID_ARG;
@@ -420,6 +462,74 @@ int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn
     r = select_into(seqs, ia, k, idx, ldi, L, ws, st);
     if (r) return r;
     return run_attn(seqs, aa, idx, ldi, k, hdr(ws), st);
+}
+
+int dsa_forward_host(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k,
+                     int32_t* idx_out, int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream,
+                     dsa_stream_t h2d_stream, dsa_stream_t d2h_stream) {
+    int r = check_seqs(seqs);
+    if (!r) r = check_indexer(seqs, ia);
+    if (!r) r = check_attn(seqs, aa);
+    if (r) return r;
+    if (!attn_is_tc(aa)) return DSA_ERR_UNSUPPORTED;
+    if (k < 1 || !packed_q_out(aa) || (idx_out && ld_idx < k)) return DSA_ERR_INVALID_ARG;
+    if (k > kTcAttnMaxSel) return DSA_ERR_UNSUPPORTED;
+    const HostLayout H = host_layout(seqs, ia, aa, k);
+    r = check_ws(ws, ws_bytes, H.total);
+    if (r) return r;
+    if (seqs->total_q == 0) return DSA_OK;
+    cudaStream_t st = (cudaStream_t)stream, sh = (cudaStream_t)h2d_stream, sd = (cudaStream_t)d2h_stream;
+    uint8_t* w = (uint8_t*)ws;
+    int32_t* idx = idx_out ? idx_out : (int32_t*)(w + H.fwd.idx);
+    const int64_t ldi = idx_out ? ld_idx : k;
+    const size_t q_row = (size_t)aa->heads * aa->dk * 2, o_row = (size_t)aa->heads * aa->dv * 2;
+
+    // events: start, Q chunk in [2], attention done [2], output chunk out [2]
+    cudaEvent_t ev[7] = {};
+    auto done = [&](int status) {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);  // released once pending work completes
+        return status;
+    };
+    for (cudaEvent_t& e : ev)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return done(DSA_ERR_CUDA);
+    cudaEvent_t ev_start = ev[0], *ev_q = ev + 1, *ev_a = ev + 3, *ev_o = ev + 5;
+    // the copy streams follow the work already queued on `stream`
+    if (cudaEventRecord(ev_start, st) != cudaSuccess || cudaStreamWaitEvent(sh, ev_start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(sd, ev_start, 0) != cudaSuccess)
+        return done(DSA_ERR_CUDA);
+    // the selection runs while the first query chunk is copied in
+    r = select_into(seqs, ia, k, idx, ldi, H.fwd, ws, st);
+    if (r) return done(r);
+    const int64_t nchunks = (seqs->total_q + H.chunk - 1) / H.chunk;
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int b = (int)(c & 1);
+        const int64_t r0 = c * H.chunk, n = (seqs->total_q - r0) < H.chunk ? (seqs->total_q - r0) : H.chunk;
+        void* qd = w + H.q[b];
+        void* od = w + H.o[b];
+        // Q in: the attention of chunk c-2 has finished reading this buffer
+        if (c >= 2 && cudaStreamWaitEvent(sh, ev_a[b], 0) != cudaSuccess) return done(DSA_ERR_CUDA);
+        if (cudaMemcpyAsync(qd, (const uint8_t*)aa->q + (size_t)r0 * q_row, (size_t)n * q_row, cudaMemcpyHostToDevice,
+                            sh) != cudaSuccess ||
+            cudaEventRecord(ev_q[b], sh) != cudaSuccess)
+            return done(DSA_ERR_CUDA);
+        // attention: Q is in, and the output copy of chunk c-2 has left this buffer
+        if (cudaStreamWaitEvent(st, ev_q[b], 0) != cudaSuccess) return done(DSA_ERR_CUDA);
+        if (c >= 2 && cudaStreamWaitEvent(st, ev_o[b], 0) != cudaSuccess) return done(DSA_ERR_CUDA);
+        r = run_attn_tc_rows(seqs, aa, idx, ldi, k, r0, n, qd, od, hdr(ws), st);
+        if (r) return done(r);
+        if (cudaEventRecord(ev_a[b], st) != cudaSuccess) return done(DSA_ERR_CUDA);
+        // output out
+        if (cudaStreamWaitEvent(sd, ev_a[b], 0) != cudaSuccess ||
+            cudaMemcpyAsync((uint8_t*)aa->out + (size_t)r0 * o_row, od, (size_t)n * o_row, cudaMemcpyDeviceToHost, sd) !=
+                cudaSuccess ||
+            cudaEventRecord(ev_o[b], sd) != cudaSuccess)
+            return done(DSA_ERR_CUDA);
+    }
+    // `stream` is ordered after the last output copies
+    for (int b = 0; b < 2 && b < nchunks; ++b)
+        if (cudaStreamWaitEvent(st, ev_o[b], 0) != cudaSuccess) return done(DSA_ERR_CUDA);
+    return done(DSA_OK);
 }
 
 int dsa_sync_status(void* ws, dsa_stream_t stream, int64_t* detail) {

@@ -171,9 +171,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     StatusHdr* st = a.st;
     volatile int* abort = &bars->abort;
 
-    // queries of this pair: t = pair + i * npairs
+    // queries of this pair: t = row_begin + pair + i * npairs
     const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int64_t nq = pair < a.total_q ? (a.total_q - pair + npairs - 1) / npairs : 0;
+    const int64_t nq = pair < a.row_count ? (a.row_count - pair + npairs - 1) / npairs : 0;
     const int nb = rank ? 5 : 4;      // 64-column blocks of K held here
     const int col0 = rank ? 256 : 0;  // first K column
     const int dv0 = rank ? 256 : 0;   // first output column
@@ -251,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         uint32_t g = 0;  // tile of the pair's whole sequence
         bool ok = true;
         for (int64_t qi = 0; ok && qi < nq; ++qi) {
-            const int64_t t = pair + qi * npairs;
+            const int64_t t = a.row_begin + pair + qi * npairs;
             const RowInfo ri = row_info(a.sv, t);
             const int32_t* irow = a.idx + t * a.ld_idx;
             const uint32_t slot = (uint32_t)(qi & 1);
@@ -299,7 +299,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                     for (int off = (int)lane * 128; off < a.k_sel * 4; off += 32 * 128) prefetch_l2(ir + off);
                 } else if (warp <= 4) {
                     const int hh = (int)(warp - 1) * 32 + (int)lane;
-                    const char* qr = (const char*)(a.q + tn * a.q_stride_tok + (int64_t)hh * a.q_stride_head + col0);
+                    const char* qr =
+                        (const char*)(a.q + (tn - a.row_begin) * a.q_stride_tok + (int64_t)hh * a.q_stride_head + col0);
                     for (int kb = 0; kb < nb; ++kb) prefetch_l2(qr + kb * 128);
                 }
             }
@@ -555,7 +556,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 // 64-column half at ((k ^ (row & 7)) << 4); read back as 4 rows x
                 // 128 bytes per instruction
                 uint8_t* stg = smem + Lay::OFF_EPI + (warp - AT_SOFT0) * 4096;
-                __nv_bfloat16* obase = a.out + t * a.out_stride_tok + (int64_t)(quad * 32) * a.out_stride_head + dv0 + ocol;
+                __nv_bfloat16* obase =
+                    a.out + (t - a.row_begin) * a.out_stride_tok + (int64_t)(quad * 32) * a.out_stride_head + dv0 + ocol;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -570,7 +572,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                     __syncwarp();
                 }
             } else {
-                uint4* dst = (uint4*)(a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol);
+                uint4* dst = (uint4*)(a.out + (t - a.row_begin) * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) dst[i] = w[i];
             }
@@ -586,7 +588,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         int64_t t_pend = 0;
         float m_pend = -INFINITY, l_pend = 0.f;
         for (int64_t qi = 0; ok && qi < nq; ++qi) {
-            const int64_t t = pair + qi * npairs;
+            const int64_t t = a.row_begin + pair + qi * npairs;
             const uint32_t slot = (uint32_t)(qi & 1);
             if (!wait_warp(smem_u32(&bars->info_full[slot]), (uint32_t)((qi >> 1) & 1), abort, st, 0x2310)) {
                 ok = false;
@@ -599,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             if (n_tiles == 0) {  // nothing selected: zero rows, lse -inf
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&bars->info_empty[slot]));
-                uint4* dst = (uint4*)(a.out + t * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol);
+                uint4* dst = (uint4*)(a.out + (t - a.row_begin) * a.out_stride_tok + (int64_t)h * a.out_stride_head + dv0 + ocol);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
                 if (rank == 0 && is_b && a.lse) a.lse[t * 128 + h] = -INFINITY;
@@ -609,7 +611,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
             // which finish a query's tiles first; every S of the earlier queries
             // has completed (this warp saw its s_full) ----
             if (!is_b) {
-                const __nv_bfloat16* qrow = a.q + t * a.q_stride_tok + (int64_t)h * a.q_stride_head + col0;
+                const __nv_bfloat16* qrow = a.q + (t - a.row_begin) * a.q_stride_tok + (int64_t)h * a.q_stride_head + col0;
                 uint4 qreg[5][8];
 #pragma unroll
                 for (int kb = 0; kb < 5; ++kb) {
@@ -836,7 +838,7 @@ static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
         return false;
     const int pairs = attn_pairs_resident<NST, VSEP, NPB, NSX>();
     if (pairs <= 0) return false;
-    const int64_t grid_pairs = a.total_q < pairs ? a.total_q : pairs;
+    const int64_t grid_pairs = a.row_count < pairs ? a.row_count : pairs;
     attn_tc_kernel<NST, VSEP, NPB, NSX><<<(unsigned)(2 * grid_pairs), AT_THREADS, Lay::SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }
@@ -848,7 +850,7 @@ static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
 #endif
 
 bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s) {
-    if (a.total_q <= 0) return true;
+    if (a.row_count <= 0) return true;
     return a.v_separate ? launch_attn_tc_t<2, true, 2, 1>(a, s)
                         : launch_attn_tc_t<DSA_ATTN_NST, false, DSA_ATTN_NPB, DSA_ATTN_NSX>(a, s);
 }

@@ -116,6 +116,10 @@ struct AttnTcArgs {
     int64_t k_stride;
     const __nv_bfloat16* v; // V rows [total_k, >= 512] (v_separate)
     int64_t v_stride;
+    // query rows [row_begin, row_begin + row_count) are processed; q and out
+    // point at row row_begin (row t at (t - row_begin) * stride_tok); idx and
+    // lse are indexed by the absolute row t
+    int64_t row_begin, row_count;
 };
 bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s);
 

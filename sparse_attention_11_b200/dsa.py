@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_INDEX = range(7)
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
-DSA_OP_FOLD, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_ATTN, DSA_OP_FORWARD = range(5)
+DSA_OP_FOLD, DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_SPARSE_ATTN, DSA_OP_FORWARD, DSA_OP_FORWARD_HOST = range(6)
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libdsa.so not built ({LIB_PATH}); run python -m sparse_attention_11_b200.build")
@@ -50,17 +50,19 @@ _lib.dsa_index_scores.argtypes = [_S, _IA, _I64, _I64, _P, _I64, _P, _SZ, _P]
 _lib.dsa_topk.argtypes = [_S, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_sparse_attn.argtypes = [_S, _AA, _P, _I64, _I32, _P, _SZ, _P]
 _lib.dsa_forward.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P]
+_lib.dsa_forward_host.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P, _P, _P]
 _lib.dsa_select.argtypes = [_S, _IA, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_select_noalloc.argtypes = [_S, _IA, _I32, _P, _I64, _P]
 _lib.dsa_sync_status.argtypes = [_P, _P, ctypes.POINTER(_I64)]
 _lib.dsa_selftest_wait_timeout.argtypes = [_P, _SZ, _I64, _P]
 for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+           "dsa_forward_host",
            "dsa_select", "dsa_select_noalloc",
            "dsa_sync_status", "dsa_selftest_wait_timeout"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk",
-            "dsa_sparse_attn", "dsa_forward", "dsa_select", "dsa_select_noalloc", "dsa_sync_status",
+            "dsa_sparse_attn", "dsa_forward", "dsa_forward_host", "dsa_select", "dsa_select_noalloc", "dsa_sync_status",
             "dsa_selftest_wait_timeout")
 
 
@@ -173,6 +175,18 @@ def dsa_topk(seqs, scores, row_begin, row_count, k, idx, ws):
 def dsa_sparse_attn(seqs, aa, idx, k_sel, ws):
     _check(_lib.dsa_sparse_attn(ctypes.byref(seqs.c), ctypes.byref(aa), _ptr(idx), idx.stride(0), k_sel, _ptr(ws),
                                 ws.numel(), _stream()), "dsa_sparse_attn")
+
+
+def dsa_forward_host(seqs, ia, aa, k, idx_out, ws, h2d_stream=None, d2h_stream=None):
+    """dsa_forward with aa's q and out in pinned host memory (see attn_args);
+    the copies run on h2d_stream / d2h_stream (torch.cuda.Stream or None for
+    the current stream), the compute on the current stream."""
+    cur = _stream()
+    sh = ctypes.c_void_p(h2d_stream.cuda_stream) if h2d_stream is not None else cur
+    sd = ctypes.c_void_p(d2h_stream.cuda_stream) if d2h_stream is not None else cur
+    _check(_lib.dsa_forward_host(ctypes.byref(seqs.c), ctypes.byref(ia), ctypes.byref(aa), k, _ptr(idx_out),
+                                 idx_out.stride(0) if idx_out is not None else 0, _ptr(ws), ws.numel(), cur, sh, sd),
+           "dsa_forward_host")
 
 
 def dsa_forward(seqs, ia, aa, k, idx_out, ws):

@@ -106,3 +106,33 @@ def test_indexer_dtype_rules(lib):
                             ctypes.byref(n)) == 0
         sizes.append(n.value)
     assert sizes[1] > sizes[0] >= 256
+
+
+def test_forward_host_validation(lib):
+    """The host-memory forward rejects non-packed or fp32 attention operands
+    and short workspaces before touching the device; its workspace holds the
+    forward's plus two staging chunks each for Q and the output."""
+    S = _fake_seqs(lib, tq=4096, tk=4096)
+    P = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    ia = lib.dsa_indexer_args(lib.DSA_E4M3, 0x100000, 0x110000, lib.DSA_BF16, 0x200000, 0x300000, 0x310000)
+    h, dk, dv = 128, 576, 512
+    packed = lib.dsa_attn_args(lib.DSA_BF16, h, dk, dv, 0x100000, h * dk, dk, 0x200000, dk, 0x200000, dk, 0.1,
+                               0x400000, h * dv, dv, None)
+    assert lib.raw_call("dsa_workspace_size", lib.DSA_OP_FORWARD, ctypes.byref(S), 2048, ctypes.byref(ia), None,
+                        ctypes.byref(n)) == 0
+    fwd = n.value
+    assert lib.raw_call("dsa_workspace_size", lib.DSA_OP_FORWARD_HOST, ctypes.byref(S), 2048, ctypes.byref(ia),
+                        ctypes.byref(packed), ctypes.byref(n)) == 0
+    chunk = 2048  # DSA_HOST_CHUNK_ROWS
+    assert n.value >= fwd + 2 * chunk * h * (dk + dv) * 2
+    ws = P(0x10000)
+    call = lambda aa, nbytes: lib.raw_call("dsa_forward_host", ctypes.byref(S), ctypes.byref(ia), ctypes.byref(aa),
+                                           2048, None, 0, ws, nbytes, None, None, None)
+    assert call(packed, 1 << 20) == lib.DSA_ERR_WORKSPACE
+    strided = lib.dsa_attn_args(lib.DSA_BF16, h, dk, dv, 0x100000, h * 640, 640, 0x200000, dk, 0x200000, dk, 0.1,
+                                0x400000, h * dv, dv, None)
+    assert call(strided, 1 << 40) == lib.DSA_ERR_INVALID_ARG
+    f32 = lib.dsa_attn_args(lib.DSA_F32, 4, 64, 64, 0x100000, 256, 64, 0x200000, 64, 0x300000, 64, 0.1,
+                            0x400000, 256, 64, None)
+    assert call(f32, 1 << 40) == lib.DSA_ERR_UNSUPPORTED

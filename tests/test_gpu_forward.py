@@ -115,3 +115,30 @@ def test_forward_prefill_l32768():
 
 def test_forward_prefill_l131072():
     _run("prefill_l131072", 256, 24, [(131072 - 128, 128), (65536, 128)])
+
+
+@pytest.mark.parametrize("name", ["prefill_l8192", "batched"])
+def test_forward_host_matches_forward(name):
+    """dsa_forward_host (query and output in pinned host memory, chunked and
+    pipelined over three streams) returns exactly dsa_forward's output, lse and
+    indices: 4 chunks at L=8192, 2 chunks for a ragged batch."""
+    wl = W.WORKLOADS[name] if name != "batched" else \
+        W.custom("prefill_b3h", (700, 1500, 129), (700, 1500, 129), base="prefill_l8192", k=300)
+    inp, prob = make(wl)
+    prob.forward()
+    prob.check("forward")
+    ref_out, ref_lse, ref_idx = prob.out.clone(), prob.lse.clone(), prob.idx.clone()
+    q_host = torch.empty(prob.q.shape, dtype=prob.q.dtype, pin_memory=True)
+    q_host.copy_(prob.q)
+    out_host = torch.full(prob.out.shape, float("nan"), dtype=prob.out.dtype, pin_memory=True)
+    lse = torch.full_like(prob.lse, float("nan"))
+    idx = torch.full_like(prob.idx, -7)
+    aa = dsa.attn_args(q_host, prob.K, prob.V, wl.scale, out_host, lse)
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD_HOST, prob.seqs, wl.k, prob.ia, aa))
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    dsa.dsa_forward_host(prob.seqs, prob.ia, aa, wl.k, idx, ws, h2d, d2h)
+    dsa.check_device_status(ws, "forward_host")
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(lse, ref_lse)
+    assert torch.equal(out_host, ref_out.cpu())
