@@ -661,15 +661,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                 const uint32_t mlo = vmask[slot * 64 + 2 * u], mhi = vmask[slot * 64 + 2 * u + 1];
                 if (!wait_warp(smem_u32(&bars->s_full), g & 1, abort, st, 0x2301)) { ok = false; break; }
                 tc_fence_after();
-                // this CTA's partial S = accumulator 0 + accumulator 1; the peer's key
-                // half first (stage A sends it on), then this CTA's own half
+                // this CTA's partial S = accumulator 0 + accumulator 1, both key
+                // halves read in one TMEM round trip; stage A sends the peer's
+                // half on before it forms the partial maximum
                 const uint32_t ta = tmem + lane_off + TM_S;
                 const int ph_ = kh ^ 1, oh = kh;  // key halves: the peer's, this CTA's
-                uint32_t rp[32], ro[32];
+                uint32_t rp[32], ro[32], xo[32];
                 {
                     uint32_t x[32];
                     tmem_ld32(ta + 32 * ph_, rp);
                     tmem_ld32(ta + 64 + 32 * ph_, x);
+                    tmem_ld32(ta + 32 * oh, ro);
+                    tmem_ld32(ta + 64 + 32 * oh, xo);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) rp[i] = __float_as_uint(__uint_as_float(rp[i]) + __uint_as_float(x[i]));
@@ -683,14 +686,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                     for (int c = 0; c < 8; ++c)
                         st_async_v4(dst + chunk_off(h, c), rp[4 * c], rp[4 * c + 1], rp[4 * c + 2], rp[4 * c + 3], bar);
                 }
-                {
-                    uint32_t x[32];
-                    tmem_ld32(ta + 32 * oh, ro);
-                    tmem_ld32(ta + 64 + 32 * oh, x);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) + __uint_as_float(x[i]));
-                }
+                for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) + __uint_as_float(xo[i]));
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
