@@ -189,8 +189,10 @@ int run_fold(const dsa_seqs* s, const dsa_indexer_args* ia, void* u, float* s_ro
     return cuda_status();
 }
 
+// fill: write -inf past each row's position (the dsa_index_scores contract;
+// the selection reads only positions 0..pos and skips it)
 int run_scores_simt(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u, const float* s_row, int64_t row_begin,
-                    int64_t row_count, float* scores, int64_t ld, StatusHdr* h, cudaStream_t st) {
+                    int64_t row_count, float* scores, int64_t ld, StatusHdr* h, cudaStream_t st, bool fill) {
     ScoresSimtArgs a;
     a.sv = seq_view(s);
     a.idx_dtype = ia->dtype;
@@ -204,6 +206,7 @@ int run_scores_simt(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u
     a.scores = scores;
     a.ld = ld;
     a.st = h;
+    a.fill = fill;
     launch_scores_simt(a, st);
     return cuda_status();
 }
@@ -387,7 +390,7 @@ int dsa_index_scores(const dsa_seqs* seqs, const dsa_indexer_args* ia, int64_t r
                               row_begin, row_count, hdr(ws), st);
     }
     return run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), row_begin, row_count, scores, ld_scores,
-                           hdr(ws), st);
+                           hdr(ws), st, true);
 }
 
 int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_scores, int64_t row_begin, int64_t row_count,
@@ -424,7 +427,7 @@ int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int
                               st);
     float* sc = (float*)(w + L.scores);
     const int64_t ld = seqs->max_seqlen_k;
-    r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st);
+    r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st, false);
     if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st);
     return r;
 }

@@ -32,6 +32,7 @@ struct ScoresSimtArgs {
     float* scores;
     int64_t ld;
     StatusHdr* st;
+    bool fill;  // write -inf to every entry past a row's position (dsa_index_scores)
 };
 void launch_scores_simt(const ScoresSimtArgs& a, cudaStream_t s);
 

@@ -16,7 +16,8 @@ namespace dsa {
 
 // ---------------------------------------------------------------------------
 // a1: fold.  Thread j of a 128-thread CTA keeps column j of W in registers
-// and folds FOLD_ROWS query rows: u_j = sum_i q_i W[i][j] (fp32 FMA chain).
+// and folds up to FOLD_ROWS query rows (fewer when there are few rows, so
+// that the CTAs cover the GPU): u_j = sum_i q_i W[i][j] (fp32 FMA chain).
 // E4M3: s_u = amax/448 (IEEE division), codes = e4m3_rn_satfinite(u_j / s_u),
 // s_row = s_q * s_u.
 // ---------------------------------------------------------------------------
@@ -30,7 +31,7 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
 __global__ void __launch_bounds__(128) fold_kernel(int64_t T, int idx_dtype, const void* __restrict__ q_idx,
                                                    const float* __restrict__ q_scale, int w_dtype,
                                                    const void* __restrict__ W, void* __restrict__ u_out,
-                                                   float* __restrict__ s_row_out) {
+                                                   float* __restrict__ s_row_out, int rows_per_cta) {
     __shared__ float qs[128];
     __shared__ float red[4];
     const int j = threadIdx.x;
@@ -42,8 +43,8 @@ __global__ void __launch_bounds__(128) fold_kernel(int64_t T, int idx_dtype, con
         else
             w[i] = __bfloat162float(((const __nv_bfloat16*)W)[i * 128 + j]);
     }
-    const int64_t r0 = (int64_t)blockIdx.x * FOLD_ROWS;
-    for (int rr = 0; rr < FOLD_ROWS; ++rr) {
+    const int64_t r0 = (int64_t)blockIdx.x * rows_per_cta;
+    for (int rr = 0; rr < rows_per_cta; ++rr) {
         const int64_t r = r0 + rr;
         if (r >= T) break;
         __syncthreads();
@@ -74,9 +75,13 @@ __global__ void __launch_bounds__(128) fold_kernel(int64_t T, int idx_dtype, con
 }
 
 void launch_fold(const FoldArgs& a, cudaStream_t s) {
-    const int64_t grid = (a.T + FOLD_ROWS - 1) / FOLD_ROWS;
-    if (grid == 0) return;
-    fold_kernel<<<(unsigned)grid, 128, 0, s>>>(a.T, a.idx_dtype, a.q_idx, a.q_scale, a.w_dtype, a.W, a.u_out, a.s_row_out);
+    if (a.T <= 0) return;
+    // about four CTAs per SM of a B200 before a CTA takes more than one row
+    int64_t rows = (a.T + 148 * 4 - 1) / (148 * 4);
+    if (rows > FOLD_ROWS) rows = FOLD_ROWS;
+    const int64_t grid = (a.T + rows - 1) / rows;
+    fold_kernel<<<(unsigned)grid, 128, 0, s>>>(a.T, a.idx_dtype, a.q_idx, a.q_scale, a.w_dtype, a.W, a.u_out, a.s_row_out,
+                                               (int)rows);
 }
 
 // ---------------------------------------------------------------------------
@@ -138,6 +143,27 @@ __global__ void __launch_bounds__(128) scores_f32_kernel(SeqView sv, const float
 // ---------------------------------------------------------------------------
 constexpr int SCAN_KEYS = 1024;
 
+// 16 e4m3 codes (one 16-byte slice of a key) dotted with 16 fp32 query
+// values: the codes are decoded in pairs by the hardware conversion to f16
+// (exact for every e4m3 value), then widened to fp32.
+__device__ __forceinline__ float dot16_e4m3(const float (&uq)[16], uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[q] >> (16 * p)), __NV_E4M3);
+            const float2 f = __half22float2(__half2(h2));
+            acc = fmaf(uq[4 * q + 2 * p], f.x, acc);
+            acc = fmaf(uq[4 * q + 2 * p + 1], f.y, acc);
+        }
+    }
+    return acc;
+}
+
+constexpr int SCAN_UNROLL = 4;  // keys per lane group in flight
+
 __global__ void __launch_bounds__(256) scan_fp8_kernel(SeqView sv, const uint8_t* __restrict__ u8,
                                                        const float* __restrict__ s_row, const uint8_t* __restrict__ k8,
                                                        const float* __restrict__ k_scale, int64_t row_begin,
@@ -160,28 +186,34 @@ __global__ void __launch_bounds__(256) scan_fp8_kernel(SeqView sv, const uint8_t
     const float srow = s_row[t];
     const int64_t s_begin = (int64_t)blockIdx.x * SCAN_KEYS;
     const int64_t s_end = min(s_begin + SCAN_KEYS, ri.pos + 1);
-    for (int64_t s0 = s_begin; s0 < s_end; s0 += 32) {
-        const int64_t s = s0 + (threadIdx.x >> 3);
-        float acc = 0.f;
-        if (s < s_end) {
-            const uint4 v = __ldg((const uint4*)(k8 + (ri.key_base + s) * 128 + sub * 16));
-            const uint8_t* b = (const uint8_t*)&v;
+    for (int64_t s0 = s_begin; s0 < s_end; s0 += 32 * SCAN_UNROLL) {
+        uint4 kv[SCAN_UNROLL];
+        float ks[SCAN_UNROLL];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc = fmaf(uq[i], e4m3_to_f32(b[i]), acc);
+        for (int u = 0; u < SCAN_UNROLL; ++u) {  // every load of the group first
+            const int64_t s = s0 + u * 32 + (threadIdx.x >> 3);
+            kv[u] = make_uint4(0u, 0u, 0u, 0u);
+            ks[u] = 0.f;
+            if (s < s_end) {
+                kv[u] = __ldg((const uint4*)(k8 + (ri.key_base + s) * 128 + sub * 16));
+                if (sub == 0) ks[u] = __ldg(k_scale + ri.key_base + s);
+            }
         }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-        if (sub == 0 && s < s_end) {
-            const float x = __fmul_rn(__fmul_rn(acc, __ldg(k_scale + ri.key_base + s)), srow);
-            scores[r * ld + s] = relu_key(x);
+#pragma unroll
+        for (int u = 0; u < SCAN_UNROLL; ++u) {
+            const int64_t s = s0 + u * 32 + (threadIdx.x >> 3);
+            float acc = dot16_e4m3(uq, kv[u]);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+            if (sub == 0 && s < s_end) scores[r * ld + s] = relu_key(__fmul_rn(__fmul_rn(acc, ks[u]), srow));
         }
     }
 }
 
 void launch_scores_simt(const ScoresSimtArgs& a, cudaStream_t s) {
     if (a.row_count <= 0) return;
-    launch_fill_neg_inf(a.scores, a.row_count, a.ld, s);
+    if (a.fill) launch_fill_neg_inf(a.scores, a.row_count, a.ld, s);
     if (a.idx_dtype == DSA_F32) {
         dim3 grid((unsigned)((a.max_seqlen_k + 127) / 128), (unsigned)a.row_count);
         scores_f32_kernel<<<grid, 128, 0, s>>>(a.sv, (const float*)a.u, (const float*)a.k_idx, a.row_begin, a.scores,
