@@ -227,11 +227,15 @@ void launch_scores_simt(const ScoresSimtArgs& a, cudaStream_t s) {
 
 // ---------------------------------------------------------------------------
 // a3: exact top-k of one row per CTA by most-significant-digit radix select
-// (4 digits of 8 bits over an order-preserving 32-bit key), then an
-// emission pass in ascending index order.  Ties at the threshold go to the
-// lowest indices.  Key order: NaN < -inf < ... < -0.0 == +0.0 < ... < +inf.
+// (4 digits of 8 bits over an order-preserving 32-bit key), then an emission
+// pass in ascending index order.  Ties at the threshold go to the lowest
+// indices.  Key order: NaN < -inf < ... < -0.0 == +0.0 < ... < +inf.  The
+// emission gives each warp a contiguous index range: the warps count their
+// keys above and in the bucket, one scan over the 32 warps gives each its
+// output offset, and each warp places its keys with ballots.
 // ---------------------------------------------------------------------------
 constexpr int TOPK_NT = 1024;
+constexpr int TOPK_WARPS = TOPK_NT / 32;
 
 __device__ __forceinline__ uint32_t order_key(float x) {
     uint32_t u = __float_as_uint(x);
@@ -240,35 +244,11 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix count of `flag` over the CTA (all TOPK_NT threads call).
-__device__ __forceinline__ int cta_excl_scan(int flag, int* warp_tot, int* total) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const unsigned bal = __ballot_sync(0xffffffffu, flag);
-    const int in_warp = __popc(bal & ((1u << lane) - 1u));
-    __syncthreads();
-    if (lane == 0) warp_tot[w] = __popc(bal);
-    __syncthreads();
-    if (w == 0) {
-        int v = warp_tot[lane];
-        int inc = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += n;
-        }
-        warp_tot[lane] = inc - v;
-        if (lane == 31) warp_tot[32] = inc;
-    }
-    __syncthreads();
-    *total = warp_tot[32];
-    return warp_tot[w] + in_warp;
-}
-
 __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld,
                                                             int64_t row_begin, int k, int32_t* __restrict__ idx,
                                                             int64_t ld_idx, StatusHdr* st) {
     __shared__ uint32_t hist[256];
-    __shared__ int warp_tot[33];
+    __shared__ uint32_t wcnt[TOPK_WARPS][2];  // per warp: keys above, keys equal (then their prefixes)
     __shared__ uint32_t sel_bin, sel_above;
     const int64_t r = blockIdx.x;
     const int64_t t = row_begin + r;
@@ -284,6 +264,7 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
         for (int64_t s = threadIdx.x; s < k; s += TOPK_NT) out[s] = s < n ? (int32_t)s : -1;
         return;
     }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t prefix = 0, mask = 0;
     uint32_t need = (uint32_t)k;
     for (int pass = 0; pass < 4; ++pass) {
@@ -335,27 +316,55 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
         __syncthreads();
         if (in_bin == need) break;
     }
-    // emission in ascending index order
-    int base_out = 0, taken = 0;
-    for (int64_t s0 = 0; s0 < n; s0 += TOPK_NT) {
-        const int64_t s = s0 + threadIdx.x;
-        int above = 0, eq = 0;
-        if (s < n) {
-            const uint32_t m = order_key(row[s]) & mask;
-            above = m > prefix;
-            eq = m == prefix;
-        }
-        int eq_total;
-        const int eq_rank = cta_excl_scan(eq, warp_tot, &eq_total);
-        const int take = above || (eq && taken + eq_rank < (int)need);
-        int take_total;
-        const int at = cta_excl_scan(take, warp_tot, &take_total);
-        if (take) out[base_out + at] = (int32_t)s;
-        base_out += take_total;
-        taken += min(eq_total, max((int)need - taken, 0));
+    // ---- emission: warp w owns indices [w*span, (w+1)*span) ----
+    const int64_t span = (((n + TOPK_WARPS - 1) / TOPK_WARPS) + 31) & ~(int64_t)31;
+    const int64_t w0 = (int64_t)warp * span, w1 = min(n, w0 + span);
+    uint32_t n_above = 0, n_eq = 0;
+    for (int64_t s = w0 + lane; s < w1; s += 32) {
+        const uint32_t m = order_key(row[s]) & mask;
+        n_above += m > prefix;
+        n_eq += m == prefix;
     }
-    for (int64_t s = base_out + threadIdx.x; s < k; s += TOPK_NT) out[s] = -1;
-    if (threadIdx.x == 0 && base_out != k) report(st, DSA_ERR_INDEX, -1000000 - t);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
+    if (lane == 0) {
+        wcnt[warp][0] = n_above;
+        wcnt[warp][1] = n_eq;
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive prefixes over the warps, in index order
+        const uint32_t a = wcnt[lane][0], e = wcnt[lane][1];
+        uint32_t ia = a, ie = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t va = __shfl_up_sync(0xffffffffu, ia, o), ve = __shfl_up_sync(0xffffffffu, ie, o);
+            if (lane >= o) ia += va, ie += ve;
+        }
+        wcnt[lane][0] = ia - a;
+        wcnt[lane][1] = ie - e;
+        if (lane == 31) sel_above = ia;  // keys above the bucket in all
+    }
+    __syncthreads();
+    uint32_t eq_before = wcnt[warp][1];
+    uint32_t pos = wcnt[warp][0] + min(eq_before, need);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t s0 = w0; s0 < w1; s0 += 32) {
+        const int64_t s = s0 + lane;
+        const uint32_t m = s < w1 ? (order_key(row[s]) & mask) : 0u;
+        const bool ab = s < w1 && m > prefix, eq = s < w1 && m == prefix;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const bool take = ab || (eq && eq_before + (uint32_t)__popc(eqm & lt) < need);
+        const uint32_t tk = __ballot_sync(0xffffffffu, take);
+        if (take && pos + (uint32_t)__popc(tk & lt) < (uint32_t)k) out[pos + __popc(tk & lt)] = (int32_t)s;
+        pos += (uint32_t)__popc(tk);
+        eq_before += (uint32_t)__popc(eqm);
+    }
+    const uint32_t total = sel_above + need;
+    for (int64_t s = total + threadIdx.x; s < k; s += TOPK_NT) out[s] = -1;
+    if (threadIdx.x == 0 && total != (uint32_t)k) report(st, DSA_ERR_INDEX, -1000000 - t);
 }
 
 void launch_topk_rows(const TopkArgs& a, cudaStream_t s) {
