@@ -227,6 +227,27 @@ void orc_topk(int64_t n, const float* scores, int64_t ld, const int64_t* ncand, 
     }
 }
 
+/* Dynamic k ([V32] §6 names a per-query k as a future direction): row r
+ * keeps K_r = min(clamp(k_rows[r], 0, k), ncand[r]) keys by the same order,
+ * written in its row of width k (ld_idx >= k) with -1 after them. */
+void orc_topk_dyn(int64_t n, const float* scores, int64_t ld, const int64_t* ncand, const int32_t* k_rows,
+                  int32_t k, int32_t* idx, int64_t ld_idx) {
+    int64_t r;
+#pragma omp parallel
+    {
+        orc_cand* buf = (orc_cand*)malloc(sizeof(orc_cand) * (size_t)(ld > 0 ? ld : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (r = 0; r < n; ++r) {
+            int32_t kr = k_rows[r] < 0 ? 0 : (k_rows[r] > k ? k : k_rows[r]);
+            int32_t* row = idx + r * ld_idx;
+            int32_t s;
+            topk_row(scores + r * ld, ncand[r], kr, buf, row);
+            for (s = kr; s < k; ++s) row[s] = -1;
+        }
+        free(buf);
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Step a4: sparse MQA attention over the selected rows ([V32] §2.3, §3.1)     */
 /* ------------------------------------------------------------------------- */

@@ -46,6 +46,7 @@ def _load():
         L.orc_fold.argtypes = [I64, I, P, P, I, P, P, P]
         L.orc_scores.argtypes = [I64, I, P, P, P, P, P, P, I64, P]
         L.orc_topk.argtypes = [I64, P, I64, P, I32, P, I64]
+        L.orc_topk_dyn.argtypes = [I64, P, I64, P, P, I32, P, I64]
         L.orc_attention.argtypes = [I64, I, I, I, I, P, P, I64, P, I64, P, P, I64, I32,
                                     ctypes.c_double, P, P]
         L.orc_forward_rows.argtypes = [I64, I, P, P, I, P, P, P, P, P, I64, I32,
@@ -120,6 +121,16 @@ def topk(scores_arr, ncand, k):
     n, ld = s.shape
     idx = np.empty((n, k), dtype=np.int32)
     _load().orc_topk(n, _p(s), ld, _p(_c(ncand, np.int64)), int(k), _p(idx), k)
+    return idx
+
+
+def topk_dyn(scores_arr, ncand, k_rows, k):
+    """Dynamic k: row r keeps min(clamp(k_rows[r], 0, k), ncand[r]) keys (same
+    order as topk), in a row of width k padded with -1."""
+    s = np.ascontiguousarray(scores_arr, dtype=np.float32)
+    n, ld = s.shape
+    idx = np.empty((n, k), dtype=np.int32)
+    _load().orc_topk_dyn(n, _p(s), ld, _p(_c(ncand, np.int64)), _p(_c(k_rows, np.int32)), int(k), _p(idx), k)
     return idx
 
 

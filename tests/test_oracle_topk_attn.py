@@ -59,6 +59,32 @@ def test_topk_brute_force_ties(seed):
             assert list(idx[r, :K]) == order[:K]
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_dynamic_k_brute_force(seed):
+    """Dynamic k (a per-query k, [V32] §6): row r keeps
+    min(clamp(k_r, 0, k), ncand_r) keys by the same order as top-k, then -1
+    up to the row width k.  Brute force with Python's sort, on tie-heavy rows,
+    with k_r of 0, 1, beyond the row, above k and negative."""
+    rng = np.random.default_rng(100 + seed)
+    n, ld, k = 40, 60, 24
+    levels = np.array([0.0, -0.0, 1.0, 2.5, 2.5, 1e-40, np.nan, 7.0, 3.0], dtype=np.float32)
+    sc = levels[rng.integers(0, len(levels), size=(n, ld))].astype(np.float32)
+    ncand = rng.integers(1, ld + 1, size=n)
+    k_rows = rng.integers(-3, k + 10, size=n).astype(np.int32)
+    k_rows[:4] = [0, 1, k, 1000]
+    idx = oracle.topk_dyn(sc, ncand, k_rows, k)
+    assert idx.shape == (n, k)
+    for r in range(n):
+        kr = min(max(int(k_rows[r]), 0), k)
+        order = sorted(range(int(ncand[r])),
+                       key=lambda s: (1, 0.0, s) if np.isnan(sc[r, s]) else (0, -float(sc[r, s]), s))
+        K = min(kr, int(ncand[r]))
+        assert list(idx[r, :K]) == order[:K]
+        assert np.all(idx[r, K:] == -1)
+    # k_r >= k everywhere is plain top-k
+    assert np.array_equal(oracle.topk_dyn(sc, ncand, np.full(n, k, np.int32), k), oracle.topk(sc, ncand, k))
+
+
 def test_topk_all_causal_when_prefix_fits():
     rng = np.random.default_rng(7)
     sc = rng.standard_normal((20, 64)).astype(np.float32)
