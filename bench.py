@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--workload", default="prefill_l32768")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dynk", action="store_true", help="skip the dynamic-k line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
     return ap.parse_args()
@@ -239,6 +240,49 @@ def run_native_workload(wl, steps, warmup, ws_n, rank, sampler=None):
     return inp, prob, ms, sel_ms, att_ms, clocks
 
 
+def dynamic_k_native(inp, prob, steps, warmup, lo=256, seed=11):
+    """Dynamic k (a per-query k): the same prefill step with k_t drawn
+    uniformly in [lo, k] per query (seeded), device-timed like the main line."""
+    import numpy as np
+    import torch
+    from sparse_attention_11_b200 import dsa
+    wl = prob.wl
+    rng = np.random.default_rng(seed)
+    kr = rng.integers(lo, wl.k + 1, size=wl.total_q).astype(np.int32)
+    ia = dsa.indexer_args(prob.q_idx, prob.q_idx_scale, prob.W, prob.k_idx, prob.k_idx_scale,
+                          k_per_row=torch.from_numpy(kr).cuda())
+    st = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(st)
+        dsa.dsa_select(prob.seqs, ia, wl.k, prob.idx, prob.ws)
+        if evs:
+            evs[1].record(st)
+        dsa.dsa_sparse_attn(prob.seqs, prob.aa, prob.idx, wl.k, prob.ws)
+        if evs:
+            evs[2].record(st)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    dsa.check_device_status(prob.ws, "dynamic k")
+    ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    pos = np.concatenate([np.arange(sk - sq, sk) for sq, sk in zip(wl.seqlens_q, wl.seqlens_k)])
+    sum_sel = int(np.minimum(kr, pos + 1).sum())
+    flops = 2.0 * wl.heads * (wl.dk + wl.dv) * sum_sel
+    return {"k_per_query": f"uniform [{lo}, {wl.k}] (seed {seed}); K_t = min(k_t, pos+1)",
+            "value": wl.total_q / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "stages_ms": {"select": sel_ms, "attention": att_ms}, "sum_selected": sum_sel,
+            "attention_tflops": flops / (att_ms / 1e3) / 1e12}
+
+
 def e2e_native(inp, prob, steps):
     """The same metric through the host-memory API, dsa_forward_host: every
     step copies its inputs from pinned host memory (the key-side tensors on the
@@ -355,6 +399,8 @@ def native(args):
     if tr:
         res["roofline"]["traffic"] = tr["bytes_per_launch"]
         res["roofline"]["traffic_source"] = tr["source"]
+    if not args.no_dynk and wl.name != "decode_b64":
+        res["dynamic_k"] = dynamic_k_native(inp, prob, max(3, min(args.steps, 10)), args.warmup)
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_native(inp, prob, max(1, min(args.steps, 5)))
         e2e_max = max_over_ranks(e2e_ms, ws_n, dev)

@@ -95,7 +95,12 @@ typedef struct dsa_seqs {
  * dtype DSA_F32:  q_idx, k_idx are float [*,128]; scales must be NULL;
  *                 w_index is DSA_F32.
  * dtype DSA_E4M3: q_idx, k_idx are e4m3 codes [*,128] with one fp32 scale
- *                 per token (value = code * scale); w_index is DSA_BF16.   */
+ *                 per token (value = code * scale); w_index is DSA_BF16.
+ * k_per_row (nullable, device int32 [total_q]): dynamic k, the per-query
+ * budget the page names as a future direction (§6).  Query t keeps
+ * K_t = min(clamp(k_per_row[t], 0, k), pos_t + 1) keys instead of
+ * min(k, pos_t + 1); the index row keeps its width k (-1 after the K_t kept
+ * keys).  NULL: every query uses k.                                        */
 typedef struct dsa_indexer_args {
     int32_t dtype;            /* DSA_F32 | DSA_E4M3 */
     const void* q_idx;        /* [total_q, 128], rows contiguous */
@@ -104,6 +109,7 @@ typedef struct dsa_indexer_args {
     const void* w_index;      /* [128, 128], W[i][j] at i*128 + j */
     const void* k_idx;        /* [total_k, 128], rows contiguous */
     const float* k_idx_scale; /* [total_k] (E4M3) */
+    const int32_t* k_per_row; /* nullable: per-query k (see above) */
 } dsa_indexer_args;
 
 /* Sparse MQA attention operands (§2.3, §3.1).
@@ -132,7 +138,8 @@ typedef struct dsa_attn_args {
 /* Human-readable name of a status code (static string). */
 DSA_API const char* dsa_status_string(int status);
 
-/* Library ABI version (major*1000 + minor). */
+/* Library ABI version (major*1000 + minor).  1001: dsa_indexer_args gained
+ * k_per_row. */
 DSA_API int dsa_version(void);
 
 /* Workspace bytes needed by `op` for this problem (k = top-k size, used by

@@ -223,6 +223,7 @@ int run_indexer_tc(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u,
     a.s_row = s_row;
     a.k_scale = ia->k_idx_scale;
     a.k = k;
+    a.k_rows = mode == 0 ? ia->k_per_row : nullptr;
     a.idx = idx;
     a.ld_idx = ld_idx;
     a.scores = scores;
@@ -239,8 +240,9 @@ int run_indexer_tc(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u,
 }
 
 int run_topk(const dsa_seqs* s, const float* scores, int64_t ld, int64_t row_begin, int64_t row_count, int32_t k,
-             int32_t* idx, int64_t ld_idx, StatusHdr* h, cudaStream_t st) {
+             int32_t* idx, int64_t ld_idx, StatusHdr* h, cudaStream_t st, const int32_t* k_rows = nullptr) {
     TopkArgs a;
+    a.k_rows = k_rows;
     a.sv = seq_view(s);
     a.scores = scores;
     a.ld = ld;
@@ -332,7 +334,7 @@ const char* dsa_status_string(int status) {
     return "unknown status";
 }
 
-int dsa_version(void) { return 1000; }
+int dsa_version(void) { return 1001; }
 
 int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexer_args* ia, const dsa_attn_args* aa,
                        size_t* bytes) {
@@ -428,7 +430,7 @@ int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int
     float* sc = (float*)(w + L.scores);
     const int64_t ld = seqs->max_seqlen_k;
     r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st, false);
-    if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st);
+    if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row);
     return r;
 }
 }  // namespace

@@ -40,7 +40,8 @@ struct TopkArgs {
     SeqView sv;
     const float* scores;
     int64_t ld, row_begin, row_count;
-    int k;
+    int k;                   // row width, and the k of rows without k_rows
+    const int32_t* k_rows;   // nullable: per-row k (clamped to [0, k]), indexed by the absolute row
     int32_t* idx;
     int64_t ld_idx;
     StatusHdr* st;
@@ -84,7 +85,8 @@ struct IndexerTcArgs {
     int64_t total_q, max_seqlen_q;
     const float* s_row;     // [total_q]
     const float* k_scale;   // [total_k]
-    int k;                  // top-k size (mode 0)
+    int k;                  // top-k size and index row width (mode 0)
+    const int32_t* k_rows;  // nullable: per-row k (clamped to [0, k])
     int32_t* idx;           // mode 0: [total_q, ld_idx]
     int64_t ld_idx;
     float* scores;          // mode 1: [row_count, ld]

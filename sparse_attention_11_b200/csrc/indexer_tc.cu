@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
     if (a.mode == 1)
         first_kind = SW_SCORES;
     else
-        first_kind = (pos_last + 1 > a.k) ? SW_HIST : SW_STOP;
+        first_kind = (pos_last + 1 > a.k || a.k_rows) ? SW_HIST : SW_STOP;
 
     const uint32_t sA = smem_u32(smem + IX_OFF_A);
     const uint32_t sB = smem_u32(smem + IX_OFF_B);
@@ -397,17 +397,23 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
         const int64_t pos = pos_first + row;
         const float srow = has_row ? __ldg(a.s_row + t) : 0.f;
         const bool in_range = a.mode != 1 || (t >= a.row_begin && t < a.row_begin + a.row_count);
-        const bool take_all = pos + 1 <= a.k;
+        // this row's k (dynamic k: clamped to [0, k]); the index row is k wide
+        const int k_row = (a.k_rows && has_row && a.mode == 0) ? min(max(__ldg(a.k_rows + t), 0), a.k) : a.k;
+        const bool take_all = pos + 1 <= k_row && k_row > 0;
         // radix state
         int level = 0;
         RowSel rs;
         rs.sh = 31;
         rs.P = 0;
-        rs.need = (uint32_t)a.k;
+        rs.need = (uint32_t)k_row;
         rs.taken = 0;
         rs.cnt = 0;
         rs.take_all = take_all;
-        bool resolved = !has_row || take_all;
+        bool resolved = !has_row || take_all || k_row == 0;
+        if (k_row == 0) {  // nothing kept: a bucket no key falls into
+            rs.P = 0x7FFFFFFF;
+            rs.sh = 31;
+        }
         uint32_t* myhist = hist + row;  // bin b at myhist[b * IX_BM]
         int32_t* out = (a.mode == 0 && has_row) ? a.idx + t * a.ld_idx : nullptr;
         float* srow_out = (a.mode == 1 && has_row && in_range) ? a.scores + (t - a.row_begin) * a.ld_scores : nullptr;
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
                 for (int64_t s = 0; s <= pos; ++s) out[s] = (int32_t)s;
                 rs.cnt = (int)(pos + 1);
             }
-            const int expect = (int)min((int64_t)a.k, pos + 1);
+            const int expect = (int)min((int64_t)k_row, pos + 1);
             if (rs.cnt != expect && !*abort) report(st, DSA_ERR_INDEX, -2000000 - t);
             for (int s = min(rs.cnt, a.k); s < a.k; ++s) out[s] = -1;
         }

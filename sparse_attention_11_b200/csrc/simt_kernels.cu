@@ -245,8 +245,8 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 }
 
 __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld,
-                                                            int64_t row_begin, int k, int32_t* __restrict__ idx,
-                                                            int64_t ld_idx, StatusHdr* st) {
+                                                            int64_t row_begin, int width, const int32_t* __restrict__ k_rows,
+                                                            int32_t* __restrict__ idx, int64_t ld_idx, StatusHdr* st) {
     __shared__ uint32_t hist[256];
     __shared__ uint32_t wcnt[TOPK_WARPS][2];  // per warp: keys above, keys equal (then their prefixes)
     __shared__ uint32_t sel_bin, sel_above;
@@ -260,8 +260,10 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
     }
     const int64_t n = ri.pos + 1;
     const float* row = scores + r * ld;
-    if (n <= k) {
-        for (int64_t s = threadIdx.x; s < k; s += TOPK_NT) out[s] = s < n ? (int32_t)s : -1;
+    // this row's k (dynamic k: clamped to [0, width]); the row is `width` wide
+    const int k = k_rows ? min(max(__ldg(k_rows + t), 0), width) : width;
+    if (n <= k || k == 0) {
+        for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = (s < n && s < k) ? (int32_t)s : -1;
         return;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -363,14 +365,14 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
         eq_before += (uint32_t)__popc(eqm);
     }
     const uint32_t total = sel_above + need;
-    for (int64_t s = total + threadIdx.x; s < k; s += TOPK_NT) out[s] = -1;
+    for (int64_t s = total + threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
     if (threadIdx.x == 0 && total != (uint32_t)k) report(st, DSA_ERR_INDEX, -1000000 - t);
 }
 
 void launch_topk_rows(const TopkArgs& a, cudaStream_t s) {
     if (a.row_count <= 0) return;
-    topk_rows_kernel<<<(unsigned)a.row_count, TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k, a.idx, a.ld_idx,
-                                                              a.st);
+    topk_rows_kernel<<<(unsigned)a.row_count, TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k, a.k_rows, a.idx,
+                                                              a.ld_idx, a.st);
 }
 
 // ---------------------------------------------------------------------------

@@ -31,7 +31,7 @@ class dsa_seqs(ctypes.Structure):
 
 class dsa_indexer_args(ctypes.Structure):
     _fields_ = [("dtype", _I32), ("q_idx", _P), ("q_idx_scale", _P), ("w_dtype", _I32), ("w_index", _P),
-                ("k_idx", _P), ("k_idx_scale", _P)]
+                ("k_idx", _P), ("k_idx_scale", _P), ("k_per_row", _P)]
 
 
 class dsa_attn_args(ctypes.Structure):
@@ -122,15 +122,17 @@ class Seqs:
         return self.c.max_seqlen_k
 
 
-def indexer_args(q_idx, q_idx_scale, w_index, k_idx, k_idx_scale):
+def indexer_args(q_idx, q_idx_scale, w_index, k_idx, k_idx_scale, k_per_row=None):
     """Indexer operands: float32 tensors (fp32 path) or uint8 e4m3 codes +
-    float32 scales with a bfloat16 W (FP8 path)."""
+    float32 scales with a bfloat16 W (FP8 path); k_per_row: optional int32
+    device tensor [total_q] of per-query k (dynamic k)."""
     fp8 = q_idx.dtype == torch.uint8
     a = dsa_indexer_args(DSA_E4M3 if fp8 else DSA_F32, q_idx.data_ptr(),
                          q_idx_scale.data_ptr() if q_idx_scale is not None else None,
                          DSA_BF16 if w_index.dtype == torch.bfloat16 else DSA_F32, w_index.data_ptr(),
-                         k_idx.data_ptr(), k_idx_scale.data_ptr() if k_idx_scale is not None else None)
-    a._keep = (q_idx, q_idx_scale, w_index, k_idx, k_idx_scale)
+                         k_idx.data_ptr(), k_idx_scale.data_ptr() if k_idx_scale is not None else None,
+                         k_per_row.data_ptr() if k_per_row is not None else None)
+    a._keep = (q_idx, q_idx_scale, w_index, k_idx, k_idx_scale, k_per_row)
     return a
 
 
