@@ -15,6 +15,11 @@ L2, so no flush is needed between steps.
 Under torchrun (N > 1) every rank runs an independent replica of the
 workload (the path shards by independent sequences; no collective on the
 data path); value = all ranks' tokens / max-over-ranks device time.
+With --cp the ranks instead split ONE sequence by query rows (context
+parallel): the key side is all-gathered over NCCL each step and value = L
+tokens / max-over-ranks time ("scaling": "strong").  At N = 1 the default
+line carries "context_parallel": the same split at 8 ranks, emulated rank
+by rank on one GPU (compute only).
 
 --impl reference times the CPU oracle (oracle/), as it stands, on the host
 cores on a bounded stratified sample of the same workload.
@@ -50,6 +55,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dynk", action="store_true", help="skip the dynamic-k line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cp", action="store_true", help="skip the emulated context-parallel line")
+    ap.add_argument("--cp", action="store_true",
+                    help="under torchrun: split one sequence over the ranks (context parallel) instead of replicas")
+    ap.add_argument("--cp-scheme", choices=["balanced", "zigzag", "contiguous"], default="balanced")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
     return ap.parse_args()
 
@@ -283,6 +292,109 @@ def dynamic_k_native(inp, prob, steps, warmup, lo=256, seed=11):
             "attention_tflops": flops / (att_ms / 1e3) / 1e12}
 
 
+def context_parallel_emulated(prob, world, schemes, steps, warmup):
+    """Context-parallel prefill with its ranks emulated in turn on this GPU.
+    Each rank's chunks run against the whole key side, which is what the
+    all-gather leaves in every rank's memory, and are timed with CUDA
+    events.  The ranks never wait on one another, so max(rank time) is the
+    compute time of a G-GPU run.  The all-gather is not timed here; its
+    bytes are reported."""
+    import torch
+    from sparse_attention_11_b200 import context_parallel as cp
+    wl = prob.wl
+    L = wl.total_q
+    st = torch.cuda.current_stream()
+    res = {"emulated_world": world, "note": "ranks run one after another on one GPU; all-gather not timed"}
+    for scheme in schemes:
+        plans = cp.plan(L, world, scheme, k=wl.k)
+        rank_ms = []
+        for chunks in plans:
+            rows = torch.cat([torch.arange(a, b) for a, b in chunks]).cuda()
+            n = rows.numel()
+            out = torch.empty((n, wl.heads, wl.dv), dtype=torch.bfloat16, device="cuda")
+            lse = torch.empty((n, wl.heads), dtype=torch.float32, device="cuda")
+            idx = torch.empty((n, wl.k), dtype=torch.int32, device="cuda")
+            run = cp.LocalForward(chunks, wl.k, prob.q_idx[rows], prob.q_idx_scale[rows], prob.W, prob.k_idx,
+                                  prob.k_idx_scale, prob.q[rows], prob.K, prob.V, wl.scale, out, lse, idx)
+            for _ in range(warmup):
+                run()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(st)
+            for _ in range(steps):
+                run()
+            e1.record(st)
+            torch.cuda.synchronize()
+            run.check("context-parallel (emulated)")
+            rank_ms.append(e0.elapsed_time(e1) / steps)
+            del run, out, lse, idx
+        mx = max(rank_ms)
+        res[scheme] = {"rank_ms": [round(x, 3) for x in rank_ms], "max_rank_ms": mx,
+                       "imbalance": mx / statistics.mean(rank_ms), "tokens_per_s_at_max_rank": L / (mx / 1e3)}
+    res["allgather_bytes_per_rank"] = int((L - L // world) * (128 + 4 + wl.dk * 2))
+    return res
+
+
+def context_parallel_native(args, ws_n, rank, dev, sampler):
+    """Context-parallel prefill on ws_n GPUs: one sequence, query rows split
+    by the plan, the key side all-gathered over NCCL every step, each rank's
+    chunks through dsa_forward.  Strong scaling: value = L tokens per step /
+    max-over-ranks device time."""
+    import torch
+    from sparse_attention_11_b200 import context_parallel as cp, workloads as W
+    from sparse_attention_11_b200.problem import DeviceProblem
+    wl = W.WORKLOADS[args.workload]
+    L = wl.total_q
+    if wl.batch != 1 or wl.idx_dtype != "e4m3" or not wl.v_in_k:
+        raise SystemExit("--cp needs a single-sequence FP8 / MLA prefill workload")
+    inp = W.generate(wl, device="cuda")
+    full = DeviceProblem(inp, with_lse=False)
+    plans = cp.plan(L, ws_n, args.cp_scheme, k=wl.k)
+    mine = plans[rank]
+    rows = torch.cat([torch.arange(a, b) for a, b in mine]).cuda()
+    n = rows.numel()
+    q_idx, q_sc, q = full.q_idx[rows], full.q_idx_scale[rows], full.q[rows]
+    k_idx_sh, k_sc_sh, kv_sh = full.k_idx[rows], full.k_idx_scale[rows], full.K[rows]
+    W_index = full.W
+    del full, inp
+    torch.cuda.empty_cache()
+    out = torch.empty((n, wl.heads, wl.dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((n, wl.heads), dtype=torch.float32, device=dev)
+    idx = torch.empty((n, wl.k), dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream()
+
+    def step():
+        cp.forward(plans, rank, wl.k, q_idx, q_sc, W_index, k_idx_sh, k_sc_sh, q, kv_sh, wl.dv, wl.scale, out, lse,
+                   idx)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    sampler.start()
+    t0.record(st)
+    for _ in range(args.steps):
+        step()
+    t1.record(st)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(ws_n)
+    ms_max = max_over_ranks(t0.elapsed_time(t1), ws_n, dev)
+    return {
+        "metric": METRIC, "value": L * args.steps / (ms_max / 1e3), "unit": "tokens/s", "n_gpus": ws_n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "dtypes": {"indexer": "e4m3", "attention": "bf16", "accumulate": "f32"}, "data": "synthetic",
+        "config": {"workload": wl.name, "batch": 1, "seq_len": L, "top_k": wl.k, "heads": wl.heads, "dk": wl.dk,
+                   "dv": wl.dv, "v": "latent part of K", "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"context-parallel x{ws_n} ({args.cp_scheme})"},
+        "allgather_bytes_per_rank": int((L - n) * (128 + 4 + wl.dk * 2)),
+        "gpu_launches": 3 * len([c for c in mine if c[1] > c[0]]) * args.steps, "clocks": clocks,
+    }
+
+
 def e2e_native(inp, prob, steps):
     """The same metric through the host-memory API, dsa_forward_host: every
     step copies its inputs from pinned host memory (the key-side tensors on the
@@ -370,6 +482,14 @@ def native(args):
     wl = W.WORKLOADS[args.workload]
     info = workload_info(wl)
     sampler = ClockSampler(torch.cuda.current_device())
+    if args.cp:
+        res = context_parallel_native(args, ws_n, rank, dev, sampler)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if ws_n > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     inp, prob, ms, sel_ms, att_ms, clocks = run_native_workload(wl, args.steps, args.warmup, ws_n, rank, sampler)
     ms_max = max_over_ranks(ms, ws_n, dev)
     tokens_per_step = info["tokens"]
@@ -407,6 +527,8 @@ def native(args):
     # dynamic k last: it writes the problem's indices and output with another selection
     if not args.no_dynk and wl.name != "decode_b64":
         res["dynamic_k"] = dynamic_k_native(inp, prob, max(3, min(args.steps, 10)), args.warmup)
+    if not args.no_cp and ws_n == 1 and wl.batch == 1 and wl.idx_dtype == "e4m3":
+        res["context_parallel"] = context_parallel_emulated(prob, 8, ("balanced", "contiguous"), 5, 2)
     if not args.no_decode and wl.name != "decode_b64":
         del prob
         torch.cuda.empty_cache()

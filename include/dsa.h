@@ -188,11 +188,24 @@ DSA_API int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_score
 DSA_API int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx,
                     int64_t ld_idx, int32_t k_sel, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
-/* Steps a1-a3 -- fold, then the fused indexer/top-k: idx (int32
+/* Steps a1-a3 -- fold, then the indexer and the top-k: idx (int32
  * [total_q, ld_idx], ld_idx >= k) receives, for every query, its
  * K_t = min(k, pos+1) selected keys in ascending index order followed by -1
- * (the selection dsa_topk makes on the scores of dsa_index_scores).  The
- * L x L scores are never written to memory.  Workspace: DSA_OP_FORWARD. */
+ * (the selection dsa_topk makes on the scores of dsa_index_scores).
+ * Workspace: DSA_OP_FORWARD.
+ *
+ * The path depends on the shapes only:
+ * - Prefill-shaped E4M3 problems run one fused tensor-core indexer / top-k
+ *   kernel, one CTA per 128 query rows of a sequence, and the scores never
+ *   reach memory.
+ * - When such a problem has fewer than 74 row blocks (ceil(max_seqlen_q /
+ *   128) x batch) over max_seqlen_k >= 8192 keys, and the score buffer
+ *   (total_q x max_seqlen_k floats) fits in 8 GiB, the selection runs in two
+ *   launches instead.  This is the case of a query chunk over a long prefix.
+ *   The first launch is a score sweep that splits each block's key range over
+ *   several CTAs; the second is the radix top-k of dsa_topk.  The scores pass
+ *   through the workspace, and the result is the same.
+ * - Decode-shaped or F32 problems use the scan + radix top-k. */
 DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
                        int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
@@ -221,8 +234,8 @@ DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t
 DSA_API int dsa_select_noalloc(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
                                int64_t ld_idx, dsa_stream_t stream);
 
-/* The whole hot path: a1 fold -> a2+a3 fused indexer/top-k (the scores stay
- * on chip) -> a4 sparse attention.  idx_out (nullable; int32
+/* The whole hot path: a1 fold -> a2+a3 indexer/top-k (as dsa_select) -> a4
+ * sparse attention.  idx_out (nullable; int32
  * [total_q, ld_idx]) receives the selected indices as dsa_topk would
  * return them for the scores of dsa_index_scores; when NULL they live in
  * the workspace. */

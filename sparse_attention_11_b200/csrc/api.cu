@@ -73,6 +73,48 @@ bool use_tc_indexer(const dsa_seqs* s, const dsa_indexer_args* ia) {
     return ia->dtype == DSA_E4M3 && s->max_seqlen_q >= kTcIndexerMinRows;
 }
 
+// The fused indexer/top-k runs one CTA per 128-row block, which covers the
+// sweeps over the block's whole key range.  With few blocks over long key
+// ranges (a query chunk over a long prefix: context-parallel ranks, chunked
+// prefill), most SMs idle and the longest block sets the time.  There the
+// selection runs as two launches instead: a tensor-core score sweep with
+// each block's key tiles split over several CTAs, then the exact radix
+// top-k per row.  Both rank the same scores exactly, so the indices are
+// identical.  The choice depends only on the shapes, so the workspace size
+// agrees with the call.
+constexpr int64_t kSplitMaxBlocks = 74;        // fewer row blocks than half the SMs
+constexpr int64_t kSplitMinKeys = 8192;        // long key ranges only
+constexpr size_t kSplitMaxScoreBytes = (size_t)8 << 30;
+
+int64_t indexer_blocks(const dsa_seqs* s) { return ((s->max_seqlen_q + 127) / 128) * (int64_t)s->batch; }
+
+bool use_split_select(const dsa_seqs* s, const dsa_indexer_args* ia) {
+    return use_tc_indexer(s, ia) && indexer_blocks(s) < kSplitMaxBlocks && s->max_seqlen_k >= kSplitMinKeys &&
+           (size_t)s->total_q * (size_t)s->max_seqlen_k * 4 <= kSplitMaxScoreBytes;
+}
+
+// the selection needs a score buffer in the workspace
+bool needs_scores(const dsa_seqs* s, const dsa_indexer_args* ia) {
+    return !use_tc_indexer(s, ia) || use_split_select(s, ia);
+}
+
+// CTAs per row block for a score sweep: about two per SM in all, each over
+// at least four 256-key tiles.
+int score_tile_splits(const dsa_seqs* s) {
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+    }
+    const int64_t blocks = indexer_blocks(s) > 0 ? indexer_blocks(s) : 1;
+    const int64_t max_tiles = (s->max_seqlen_k + 255) / 256;
+    int64_t n = (2 * sms + blocks - 1) / blocks;
+    const int64_t cap = max_tiles / 4 > 1 ? max_tiles / 4 : 1;
+    if (n > cap) n = cap;
+    if (n > 64) n = 64;
+    return n < 1 ? 1 : (int)n;
+}
+
 struct WsLayout {
     size_t u, s_row, idx, scores, total;
 };
@@ -103,7 +145,7 @@ struct HostLayout {
 
 HostLayout host_layout(const dsa_seqs* s, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k) {
     HostLayout H;
-    H.fwd = ws_layout(s, ia, k, true, !use_tc_indexer(s, ia));
+    H.fwd = ws_layout(s, ia, k, true, needs_scores(s, ia));
     H.chunk = s->total_q < DSA_HOST_CHUNK_ROWS ? s->total_q : DSA_HOST_CHUNK_ROWS;
     H.q_chunk_bytes = (size_t)H.chunk * (size_t)aa->heads * (size_t)aa->dk * 2;
     H.o_chunk_bytes = (size_t)H.chunk * (size_t)aa->heads * (size_t)aa->dv * 2;
@@ -230,6 +272,7 @@ int run_indexer_tc(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u,
     a.ld_scores = ld_scores;
     a.row_begin = row_begin;
     a.row_count = row_count;
+    a.tile_splits = mode == 1 ? score_tile_splits(s) : 1;
     a.st = h;
     if (!make_map_2d(&a.tm_u, CU_TENSOR_MAP_DATA_TYPE_UINT8, u, 128, (uint64_t)s->total_q, 128, 128, 128))
         return DSA_ERR_CUDA;
@@ -351,7 +394,7 @@ int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexe
             return DSA_OK;
         case DSA_OP_FORWARD:
             if (!ia || k < 1) return DSA_ERR_INVALID_ARG;
-            *bytes = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia)).total;
+            *bytes = ws_layout(seqs, ia, k, true, needs_scores(seqs, ia)).total;
             return DSA_OK;
         case DSA_OP_FORWARD_HOST:
             if (!ia || !aa || k < 1 || aa->heads < 1 || aa->dk < 1 || aa->dv < 1) return DSA_ERR_INVALID_ARG;
@@ -424,11 +467,18 @@ int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int
     uint8_t* w = (uint8_t*)ws;
     int r = run_fold(seqs, ia, w + L.u, (float*)(w + L.s_row), st);
     if (r) return r;
+    float* sc = (float*)(w + L.scores);
+    const int64_t ld = seqs->max_seqlen_k;
+    if (use_split_select(seqs, ia)) {
+        // scores past each row's position are left unwritten: the top-k reads 0..pos
+        r = run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 1, 0, nullptr, 0, sc, ld, 0, seqs->total_q,
+                           hdr(ws), st);
+        if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row);
+        return r;
+    }
     if (use_tc_indexer(seqs, ia))
         return run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, k, idx, ldi, nullptr, 0, 0, 0, hdr(ws),
                               st);
-    float* sc = (float*)(w + L.scores);
-    const int64_t ld = seqs->max_seqlen_k;
     r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st, false);
     if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row);
     return r;
@@ -441,7 +491,7 @@ int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int3
     if (!r) r = check_indexer(seqs, ia);
     if (r) return r;
     if (k < 1 || (seqs->total_q && (!idx || ld_idx < k))) return DSA_ERR_INVALID_ARG;
-    const WsLayout L = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia));
+    const WsLayout L = ws_layout(seqs, ia, k, true, needs_scores(seqs, ia));
     r = check_ws(ws, ws_bytes, L.total);
     if (r) return r;
     if (seqs->total_q == 0) return DSA_OK;
@@ -457,7 +507,7 @@ int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn
     if (k < 1) return DSA_ERR_INVALID_ARG;
     if (attn_is_tc(aa) && k > kTcAttnMaxSel) return DSA_ERR_UNSUPPORTED;
     if (idx_out && ld_idx < k) return DSA_ERR_INVALID_ARG;
-    const WsLayout L = ws_layout(seqs, ia, k, true, !use_tc_indexer(seqs, ia));
+    const WsLayout L = ws_layout(seqs, ia, k, true, needs_scores(seqs, ia));
     r = check_ws(ws, ws_bytes, L.total);
     if (r) return r;
     if (seqs->total_q == 0) return DSA_OK;

@@ -91,6 +91,7 @@ struct IndexerTcArgs {
     int64_t ld_idx;
     float* scores;          // mode 1: [row_count, ld]
     int64_t ld_scores, row_begin, row_count;
+    int tile_splits;        // mode 1: CTAs per row block, each over a contiguous range of key tiles
     StatusHdr* st;
     CUtensorMap tm_u;       // folded query codes [total_q,128], box 128x128
     CUtensorMap tm_k;       // key codes [total_k,128], box 128x256

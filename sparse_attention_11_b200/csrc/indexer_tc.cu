@@ -256,10 +256,19 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
     StatusHdr* st = a.st;
     volatile int* abort = &bars->abort;
 
-    // ---- block -> (sequence, row range); heaviest blocks launch first ----
+    // ---- block -> (sequence, row range, key-tile split); heaviest blocks
+    // launch first.  Score sweeps (mode 1) may split a row block's key tiles
+    // over tile_splits CTAs, each taking a contiguous range of tiles ----
+    const int nsplit = a.tile_splits > 1 ? a.tile_splits : 1;
+    if (nsplit > 1 && a.mode != 1) {
+        if (threadIdx.x == 0) report(a.st, DSA_ERR_UNSUPPORTED, -5);
+        return;
+    }
+    const int split = (int)(blockIdx.x % nsplit);
+    const int64_t bid = (int64_t)(blockIdx.x / nsplit);
     const int64_t nblk = (a.max_seqlen_q + IX_BM - 1) / IX_BM;
-    const int b = (int)(blockIdx.x % a.sv.batch);
-    const int64_t jb = nblk - 1 - (int64_t)(blockIdx.x / a.sv.batch);
+    const int b = (int)(bid % a.sv.batch);
+    const int64_t jb = nblk - 1 - bid / a.sv.batch;
     const int64_t q0 = __ldg(a.sv.cu_q + b), sq = __ldg(a.sv.cu_q + b + 1) - q0;
     const int64_t key_base = __ldg(a.sv.cu_k + b), sk = __ldg(a.sv.cu_k + b + 1) - key_base;
     const int64_t i0 = jb * IX_BM;
@@ -274,6 +283,9 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
     const int64_t t_first = q0 + i0;
     if (a.mode == 1 && (t_first + nrows <= a.row_begin || t_first >= a.row_begin + a.row_count)) return;
     const int n_tiles = (int)((pos_last + IX_BN) / IX_BN);
+    const int per_split = (n_tiles + nsplit - 1) / nsplit;
+    const int t_lo = split * per_split, t_hi = min(n_tiles, t_lo + per_split);  // this CTA's key tiles
+    if (t_lo >= t_hi) return;
     int first_kind;
     if (a.mode == 1)
         first_kind = SW_SCORES;
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
             for (int i = 0; i < IX_NST; ++i) last_issued[i] = 0xFFFFFFFFu;
             int kind = first_kind;
             for (int sw = 0; kind != SW_STOP; ++sw) {
-                for (int tile = 0; tile < n_tiles; ++tile, ++g) {
+                for (int tile = t_lo; tile < t_hi; ++tile, ++g) {
                     const uint32_t s = g % IX_NST;
                     if (!wait_warp(smem_u32(&bars->empty[s]), ((g / IX_NST) & 1) ^ 1, abort, st, 0x1101)) break;
                     const int64_t kr0 = key_base + (int64_t)tile * IX_BN;
@@ -361,7 +373,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
             uint32_t g = 0;
             int kind = first_kind;
             for (int sw = 0; ok && kind != SW_STOP; ++sw) {
-                for (int tile = 0; tile < n_tiles; ++tile, ++g) {
+                for (int tile = t_lo; tile < t_hi; ++tile, ++g) {
                     const uint32_t s = g % IX_NST, ab = g & 1;
                     if (!wait_warp(smem_u32(&bars->full[s]), (g / IX_NST) & 1, abort, st, 0x1202)) { ok = false; break; }
                     if (!wait_warp(smem_u32(&bars->acc_empty[ab]), ((g >> 1) & 1) ^ 1, abort, st, 0x1203)) { ok = false; break; }
@@ -424,7 +436,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
         int kind = first_kind;
         for (int sw = 0; kind != SW_STOP; ++sw) {
             const int lvl = level + 1;  // histogram level of this sweep (HIST)
-            for (int tile = 0; tile < n_tiles; ++tile, ++g) {
+            for (int tile = t_lo; tile < t_hi; ++tile, ++g) {
                 const uint32_t s = g % IX_NST, ab = g & 1;
                 bool ok = wait_warp(smem_u32(&bars->acc_full[ab]), (g >> 1) & 1, abort, st, 0x1301);
                 ok = ok && wait_warp(smem_u32(&bars->full[s]), (g / IX_NST) & 1, abort, st, 0x1302);
@@ -509,8 +521,9 @@ bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s) {
     if (cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM) != cudaSuccess)
         return false;
     const int64_t nblk = (a.max_seqlen_q + IX_BM - 1) / IX_BM;
-    const int64_t grid = nblk * a.sv.batch;
+    const int64_t grid = nblk * a.sv.batch * (a.tile_splits > 1 ? a.tile_splits : 1);
     if (grid <= 0) return true;
+    if (grid >= ((int64_t)1 << 31)) return false;
     indexer_tc_kernel<<<(unsigned)grid, IX_THREADS, IX_SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }

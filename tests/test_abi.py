@@ -108,6 +108,31 @@ def test_indexer_dtype_rules(lib):
     assert sizes[1] > sizes[0] >= 256
 
 
+def test_selection_path_workspace(lib):
+    """The selection path follows from the shapes alone, and so does the
+    workspace.  Few 128-row blocks over >= 8192 keys select in two launches
+    through a score buffer of total_q x max_seqlen_k floats.  Otherwise the
+    prefill-shaped problem runs fused, with no score buffer."""
+    n = ctypes.c_size_t(0)
+    ia = lib.dsa_indexer_args(lib.DSA_E4M3, 0x100000, 0x110000, lib.DSA_BF16, 0x200000, 0x300000, 0x310000)
+
+    def size(batch, tq, tk, mq, mk):
+        S = lib.dsa_seqs(batch, tq, tk, mq, mk, 0x1000, 0x2000)
+        assert lib.raw_call("dsa_workspace_size", lib.DSA_OP_FORWARD, ctypes.byref(S), 2048, ctypes.byref(ia), None,
+                            ctypes.byref(n)) == 0
+        return n.value
+
+    k = 2048
+    split = [(1, 2048, 32768, 2048, 32768), (1, 8192, 8192, 8192, 8192), (1, 9344, 9344, 9344, 9344),
+             (2, 8192, 32768, 4096, 16384)]
+    fused = [(1, 32768, 32768, 32768, 32768), (1, 4096, 4096, 4096, 4096), (1, 9472, 9472, 9472, 9472),
+             (2, 8192, 8192, 4096, 4096)]
+    for b, tq, tk, mq, mk in split:
+        assert size(b, tq, tk, mq, mk) >= tq * mk * 4 + tq * k * 4, (b, tq, tk)
+    for b, tq, tk, mq, mk in fused:
+        assert size(b, tq, tk, mq, mk) < tq * k * 4 + tq * 256 + (1 << 20), (b, tq, tk)
+
+
 def test_forward_host_validation(lib):
     """The host-memory forward rejects non-packed or fp32 attention operands
     and short workspaces before touching the device; its workspace holds the

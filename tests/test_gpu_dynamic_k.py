@@ -2,9 +2,13 @@
 dynamic k as a future direction), through the C ABI.
 
 Query t keeps K_t = min(clamp(k_t, 0, k), pos_t + 1) keys.  Checked on the
-fused tensor-core indexer (prefill_l8192) and on the scan + radix top-k path
-(decode_b64), with per-query k drawn uniformly in [0, k] plus the edge values
-0, 1, k and past k:
+three selection paths, with per-query k drawn uniformly in [0, k] plus the
+edge values 0, 1, k and past k:
+  * prefill_l32768: the fused tensor-core indexer / top-k;
+  * prefill_l8192: 64 row blocks over 8192 keys, which selects in two
+    launches (split tensor-core score sweep, then the radix top-k);
+  * decode_b64: the scan + radix top-k.
+Each is checked as follows:
   * the fused selection equals, bit for bit, the exact top-K_t of the GPU's
     own scores (dsa_index_scores ranked by the oracle's top-k), in ascending
     order, -1 after;
@@ -33,7 +37,7 @@ def _k_rows(T, k, seed):
     return kr
 
 
-@pytest.mark.parametrize("name", ["prefill_l8192", "decode_b64"])
+@pytest.mark.parametrize("name", ["prefill_l32768", "prefill_l8192", "decode_b64"])
 def test_dynamic_k(name):
     wl = W.WORKLOADS[name]
     inp, prob = make(wl)

@@ -1,6 +1,9 @@
-"""End-to-end parity of dsa_forward (the fused path) on the five workloads.
+"""End-to-end parity of dsa_forward on the five workloads.
 
-For every checked row: the fused selection equals dsa_topk applied to the
+The selection runs fused (one tensor-core indexer / top-k kernel) at 32K and
+128K and on short sequences.  prefill_l8192 (64 row blocks over 8192 keys)
+takes the two-launch path: a key-split score sweep, then the radix top-k.
+For every checked row: the selection equals dsa_topk applied to the
 scores of dsa_index_scores (same arithmetic, bit-exact), its overlap with
 the oracle's own selection is >= 0.999, and the attention output matches the
 oracle run on the GPU's selected indices (2e-2 abs bf16, 1e-5 abs fp32).
