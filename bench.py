@@ -528,7 +528,7 @@ def native(args):
     if not args.no_dynk and wl.name != "decode_b64":
         res["dynamic_k"] = dynamic_k_native(inp, prob, max(3, min(args.steps, 10)), args.warmup)
     if not args.no_cp and ws_n == 1 and wl.batch == 1 and wl.idx_dtype == "e4m3":
-        res["context_parallel"] = context_parallel_emulated(prob, 8, ("balanced", "contiguous"), 5, 2)
+        res["context_parallel"] = context_parallel_emulated(prob, 8, ("balanced", "zigzag", "contiguous"), 5, 2)
     if not args.no_decode and wl.name != "decode_b64":
         del prob
         torch.cuda.empty_cache()

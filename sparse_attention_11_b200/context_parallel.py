@@ -39,10 +39,13 @@ from . import dsa
 
 
 # Indexer cost of one (query, key) pair relative to the attention's cost of
-# one selected key, from the measured stage times at L = 32K on a B200
-# (fused indexer + top-k 3.77 ms over 5.4e8 causal pairs; attention 28.0 ms
-# over 6.5e7 selected keys).
-INDEXER_PAIR_COST = 0.0163
+# one selected key, for a rank's chunks.  Measured on a B200 from ranks
+# emulated at L = 32K, G = 8, contiguous plan: the selection of a chunk over
+# a long prefix takes the key-split path at about 1.25e-11 s per causal
+# pair, and the attention about 4.5e-10 s per selected key.  A one-GPU run
+# of the whole sequence, whose fused selection is faster per pair, is not
+# what this plan balances.
+INDEXER_PAIR_COST = 0.028
 
 
 def row_cost(pos, k, alpha=INDEXER_PAIR_COST):

@@ -82,8 +82,8 @@ bool use_tc_indexer(const dsa_seqs* s, const dsa_indexer_args* ia) {
 // top-k per row.  Both rank the same scores exactly, so the indices are
 // identical.  The choice depends only on the shapes, so the workspace size
 // agrees with the call.
-constexpr int64_t kSplitMaxBlocks = 74;        // fewer row blocks than half the SMs
-constexpr int64_t kSplitMinKeys = 8192;        // long key ranges only
+constexpr int64_t kSplitMaxBlocks = 148;       // fewer row blocks than SMs (measured crossover on B200)
+constexpr int64_t kSplitMinKeys = 2049;        // key ranges longer than 2048 (shorter ones need few sweeps)
 constexpr size_t kSplitMaxScoreBytes = (size_t)8 << 30;
 
 int64_t indexer_blocks(const dsa_seqs* s) { return ((s->max_seqlen_q + 127) / 128) * (int64_t)s->batch; }

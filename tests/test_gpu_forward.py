@@ -1,8 +1,10 @@
 """End-to-end parity of dsa_forward on the five workloads.
 
 The selection runs fused (one tensor-core indexer / top-k kernel) at 32K and
-128K and on short sequences.  prefill_l8192 (64 row blocks over 8192 keys)
-takes the two-launch path: a key-split score sweep, then the radix top-k.
+128K and on the batched case (sequences of at most 2048 keys).  prefill_l8192
+and the 3000-token case (fewer 128-row blocks than SMs over more than 2048
+keys) take the two-launch path: a key-split score sweep, then the radix
+top-k.
 For every checked row: the selection equals dsa_topk applied to the
 scores of dsa_index_scores (same arithmetic, bit-exact), its overlap with
 the oracle's own selection is >= 0.999, and the attention output matches the
