@@ -206,6 +206,16 @@ def captured_traffic(workload, kernel):
     return tr.get(workload, {}).get(kernel)
 
 
+def step_launches(wl):
+    """Kernel launches of one prefill step (dsa_select + dsa_sparse_attn),
+    by the library's selection rule (include/dsa.h, dsa_select).  The fused
+    path is fold, indexer/top-k.  Fewer 128-row blocks than SMs over more
+    than 2048 keys add one launch: fold, score sweep, radix top-k."""
+    blocks = wl.batch * ((max(wl.seqlens_q) + 127) // 128)
+    split = max(wl.seqlens_q) >= 64 and blocks < 148 and max(wl.seqlens_k) > 2048
+    return (4 if split else 3)
+
+
 def run_native_workload(wl, steps, warmup, ws_n, rank, sampler=None):
     """Device-timed steps of select + attention on one workload."""
     import torch
@@ -512,7 +522,7 @@ def native(args):
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved_tf / peak,
                      "peak_kind": f"bf16 {peaks['source']} sustained", "flops_per_launch": flops,
                      "frac_of_burst": achieved_tf / peaks["bf16_tflops"], "traffic": None},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": step_launches(wl) * args.steps,
         "clocks": clocks,
     }
     tr = captured_traffic(wl.name, "attn_tc_kernel")
