@@ -148,9 +148,19 @@ __device__ __forceinline__ void ep_chunk(uint32_t (&v)[32], const float* scs, fl
         }
     } else if (MODE == 3) {
         if (srow_out) {
+            float* dst = srow_out + sbase;
+            if (limmask == 0xFFFFFFFFu && (((uintptr_t)dst) & 15) == 0) {
+                // a whole, aligned chunk: eight 16-byte stores instead of 32
+                // scalar ones, so the next TMEM load into v[] waits less
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if ((limmask >> i) & 1u) srow_out[sbase + i] = __int_as_float(KB(i));
+                for (int q = 0; q < 8; ++q)
+                    ((float4*)dst)[q] = make_float4(__int_as_float(KB(4 * q)), __int_as_float(KB(4 * q + 1)),
+                                                    __int_as_float(KB(4 * q + 2)), __int_as_float(KB(4 * q + 3)));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if ((limmask >> i) & 1u) dst[i] = __int_as_float(KB(i));
+            }
         }
     }
 }
@@ -246,6 +256,10 @@ __device__ __forceinline__ void ep_emit_half(uint32_t taddr, bool ok, bool activ
     rs.taken += t0 + t1;
 }
 
+// KMODE 0: the fused selection (index rows out); KMODE 1: the score sweep
+// (scores out, optionally split over key tiles).  Each mode is its own
+// instantiation, so neither carries the other's epilogue code.
+template <int KMODE>
 __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_constant__ IndexerTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
     // launch first.  Score sweeps (mode 1) may split a row block's key tiles
     // over tile_splits CTAs, each taking a contiguous range of tiles ----
     const int nsplit = a.tile_splits > 1 ? a.tile_splits : 1;
-    if (nsplit > 1 && a.mode != 1) {
+    if (nsplit > 1 && KMODE != 1) {
         if (threadIdx.x == 0) report(a.st, DSA_ERR_UNSUPPORTED, -5);
         return;
     }
@@ -281,13 +295,13 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
         return;
     }
     const int64_t t_first = q0 + i0;
-    if (a.mode == 1 && (t_first + nrows <= a.row_begin || t_first >= a.row_begin + a.row_count)) return;
+    if (KMODE == 1 && (t_first + nrows <= a.row_begin || t_first >= a.row_begin + a.row_count)) return;
     const int n_tiles = (int)((pos_last + IX_BN) / IX_BN);
     const int per_split = (n_tiles + nsplit - 1) / nsplit;
     const int t_lo = split * per_split, t_hi = min(n_tiles, t_lo + per_split);  // this CTA's key tiles
     if (t_lo >= t_hi) return;
     int first_kind;
-    if (a.mode == 1)
+    if (KMODE == 1)
         first_kind = SW_SCORES;
     else
         first_kind = (pos_last + 1 > a.k || a.k_rows) ? SW_HIST : SW_STOP;
@@ -408,9 +422,9 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
         const int64_t t = t_first + row;
         const int64_t pos = pos_first + row;
         const float srow = has_row ? __ldg(a.s_row + t) : 0.f;
-        const bool in_range = a.mode != 1 || (t >= a.row_begin && t < a.row_begin + a.row_count);
+        const bool in_range = KMODE != 1 || (t >= a.row_begin && t < a.row_begin + a.row_count);
         // this row's k (dynamic k: clamped to [0, k]); the index row is k wide
-        const int k_row = (a.k_rows && has_row && a.mode == 0) ? min(max(__ldg(a.k_rows + t), 0), a.k) : a.k;
+        const int k_row = (KMODE == 0 && a.k_rows && has_row) ? min(max(__ldg(a.k_rows + t), 0), a.k) : a.k;
         const bool take_all = pos + 1 <= k_row && k_row > 0;
         // radix state
         int level = 0;
@@ -427,8 +441,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
             rs.sh = 31;
         }
         uint32_t* myhist = hist + row;  // bin b at myhist[b * IX_BM]
-        int32_t* out = (a.mode == 0 && has_row) ? a.idx + t * a.ld_idx : nullptr;
-        float* srow_out = (a.mode == 1 && has_row && in_range) ? a.scores + (t - a.row_begin) * a.ld_scores : nullptr;
+        int32_t* out = (KMODE == 0 && has_row) ? a.idx + t * a.ld_idx : nullptr;
+        float* srow_out = (KMODE == 1 && has_row && in_range) ? a.scores + (t - a.row_begin) * a.ld_scores : nullptr;
         for (int i = 128 * half; i < 128 * half + 128; ++i) myhist[i * IX_BM] = 0;
         asm volatile("bar.sync 1, 256;" ::: "memory");  // both halves cleared the row's bins
 
@@ -445,16 +459,18 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
                 const int64_t s_tile = (int64_t)tile * IX_BN + 128 * half;
                 const bool active = ok && has_row && !(kind == SW_HIST && resolved);
                 const uint32_t taddr = tmem + ((quad * 32) << 16) + ab * IX_BN + 128 * half;
-                if (kind == SW_HIST && lvl == 1)
-                    ep_tile<1>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
-                else if (kind == SW_HIST)
-                    ep_tile<4>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, lvl == 2 ? 15 : lvl == 3 ? 7 : 0,
-                               lvl == 4 ? 127u : 255u, out, a.k, srow_out);
-                else if (kind == SW_EMIT)
-                    ep_emit_half(taddr, ok, active, scs, srow, pos, s_tile, half, rs, out, a.k,
-                                 (uint2*)(smem + IX_OFF_ECNT) + (tile & 1) * 2 * IX_BM + row, 2 + (int)quad);
-                else
+                if constexpr (KMODE == 1) {
                     ep_tile<3>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
+                } else {
+                    if (kind == SW_HIST && lvl == 1)
+                        ep_tile<1>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, 0, 0, out, a.k, srow_out);
+                    else if (kind == SW_HIST)
+                        ep_tile<4>(taddr, ok, active, scs, srow, pos, s_tile, rs, myhist, lvl == 2 ? 15 : lvl == 3 ? 7 : 0,
+                                   lvl == 4 ? 127u : 255u, out, a.k, srow_out);
+                    else if (kind == SW_EMIT)
+                        ep_emit_half(taddr, ok, active, scs, srow, pos, s_tile, half, rs, out, a.k,
+                                     (uint2*)(smem + IX_OFF_ECNT) + (tile & 1) * 2 * IX_BM + row, 2 + (int)quad);
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -501,7 +517,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
             kind = *(volatile int*)&bars->next_kind;
         }
         // ---- finish the index rows ----
-        if (a.mode == 0 && has_row && half == 0) {
+        if (KMODE == 0 && has_row && half == 0) {
             if (first_kind == SW_STOP) {  // every row of the block keeps its whole prefix
                 for (int64_t s = 0; s <= pos; ++s) out[s] = (int32_t)s;
                 rs.cnt = (int)(pos + 1);
@@ -518,13 +534,17 @@ __global__ void __launch_bounds__(IX_THREADS, 1) indexer_tc_kernel(const __grid_
 }
 
 bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s) {
-    if (cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM) != cudaSuccess)
-        return false;
+    if (a.mode != 0 && a.mode != 1) return false;
+    const void* fn = a.mode == 1 ? (const void*)indexer_tc_kernel<1> : (const void*)indexer_tc_kernel<0>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM) != cudaSuccess) return false;
     const int64_t nblk = (a.max_seqlen_q + IX_BM - 1) / IX_BM;
     const int64_t grid = nblk * a.sv.batch * (a.tile_splits > 1 ? a.tile_splits : 1);
     if (grid <= 0) return true;
     if (grid >= ((int64_t)1 << 31)) return false;
-    indexer_tc_kernel<<<(unsigned)grid, IX_THREADS, IX_SMEM, s>>>(a);
+    if (a.mode == 1)
+        indexer_tc_kernel<1><<<(unsigned)grid, IX_THREADS, IX_SMEM, s>>>(a);
+    else
+        indexer_tc_kernel<0><<<(unsigned)grid, IX_THREADS, IX_SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess;
 }
 
