@@ -38,24 +38,27 @@ import torch
 from . import dsa
 
 
-# Indexer cost of one (query, key) pair relative to the attention's cost of
-# one selected key, for a rank's chunks.  Measured on a B200 from ranks
-# emulated at L = 32K, G = 8, contiguous plan: the selection of a chunk over
-# a long prefix takes the key-split path at about 1.25e-11 s per causal
-# pair, and the attention about 4.5e-10 s per selected key.  A one-GPU run
-# of the whole sequence, whose fused selection is faster per pair, is not
-# what this plan balances.
-INDEXER_PAIR_COST = 0.028
+# Modelled cost of a rank's rows, in units of the attention's cost of one
+# selected key.  The three terms are fitted by least squares to 24 measured
+# rank times (3 plans x 8 ranks, L = 32K, ranks emulated on a B200; RMS
+# residual 0.1 ms of about 4.4 ms):
+#   0.395 ns per selected key (attention);
+#   54.6 ns per query row, 138 keys' worth (the per-query work of the
+#     attention and the selection);
+#   7.45e-12 s per causal (query, key) pair, 0.0189 keys' worth (the
+#     key-split selection that a rank's chunks take).
+INDEXER_PAIR_COST = 0.0189
+ROW_OVERHEAD = 138.0
 
 
-def row_cost(pos, k, alpha=INDEXER_PAIR_COST):
-    """Modelled cost of query rows at positions `pos`: the attention's
-    min(k, pos+1) selected keys plus alpha per causal indexer pair."""
+def row_cost(pos, k, alpha=INDEXER_PAIR_COST, overhead=ROW_OVERHEAD):
+    """Modelled cost of query rows at positions `pos`: min(k, pos+1)
+    selected keys, a per-row overhead, and alpha per causal indexer pair."""
     pos = np.asarray(pos, dtype=np.float64)
-    return np.minimum(float(k), pos + 1.0) + alpha * (pos + 1.0)
+    return np.minimum(float(k), pos + 1.0) + overhead + alpha * (pos + 1.0)
 
 
-def plan(L, world, scheme="zigzag", k=2048, alpha=INDEXER_PAIR_COST):
+def plan(L, world, scheme="zigzag", k=2048, alpha=INDEXER_PAIR_COST, overhead=ROW_OVERHEAD):
     """Chunks of query rows per rank: a list (rank) of lists of (begin, end),
     in the order the rank stores its rows.
 
@@ -70,7 +73,7 @@ def plan(L, world, scheme="zigzag", k=2048, alpha=INDEXER_PAIR_COST):
     if scheme == "zigzag":
         b = [(i * L) // n for i in range(n + 1)]
     elif scheme == "balanced":
-        c = np.concatenate([[0.0], np.cumsum(row_cost(np.arange(L), k, alpha))])
+        c = np.concatenate([[0.0], np.cumsum(row_cost(np.arange(L), k, alpha, overhead))])
         half = L // 2
         first = [c[half] * j / world for j in range(world + 1)]
         second = [c[half] + (c[L] - c[half]) * j / world for j in range(1, world + 1)]

@@ -58,14 +58,20 @@ def test_plans_balance_cost(world):
     assert ix.max() / ix.min() < 1.001  # the indexer's O(pos) cost, exactly even
     ixc, _ = _costs(cp.plan(L, world, "contiguous"), k)
     assert ixc.max() / ixc.min() > 2.0  # what zigzag removes
-    # the modelled total, attention + indexer, is even under "balanced" only
-    a = cp.INDEXER_PAIR_COST
-    tot = lambda p: (lambda i, t: t + a * i)(*_costs(p, k))
+    # the modelled total (attention keys + per-row overhead + indexer pairs)
+    # is even under "balanced" only
+    a, o = cp.INDEXER_PAIR_COST, cp.ROW_OVERHEAD
+    rows = lambda p: np.array([cp.local_rows(c) for c in p], dtype=np.float64)
+    tot = lambda p: (lambda i, t: t + a * i)(*_costs(p, k)) + o * rows(p)
     tb = tot(cp.plan(L, world, "balanced"))
     assert tb.max() / tb.min() < 1.005
     tz = tot(cp.plan(L, world, "zigzag"))
-    assert tz.max() / tz.min() > 1.05
+    assert tz.max() / tz.min() > 1.03
     assert np.isclose(tb.sum(), tz.sum())
+    # row_cost is that model, row by row
+    p = cp.plan(L, world, "balanced")
+    direct = np.array([sum(cp.row_cost(np.arange(s, e), k).sum() for s, e in c) for c in p])
+    assert np.allclose(direct, tb)
 
 
 def test_chunk_positions():
