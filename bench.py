@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--cp", action="store_true",
                     help="under torchrun: split one sequence over the ranks (context parallel) instead of replicas")
     ap.add_argument("--cp-scheme", choices=["balanced", "zigzag", "contiguous"], default="balanced")
+    ap.add_argument("--bwd", action="store_true",
+                    help="also time the sparse attention's backward (dsa_sparse_attn_bwd) on the workload")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
     return ap.parse_args()
 
@@ -405,6 +407,44 @@ def context_parallel_native(args, ws_n, rank, dev, sampler):
     }
 
 
+def backward_native(prob, steps, warmup, seed=23):
+    """The sparse attention's backward over the forward's own selection,
+    output and lse, with a seeded bf16 d_out; the MLA-tied gradient (d_V is
+    d_K's first dv columns).  Device-timed per call; d_K is zeroed between
+    calls outside the timed region."""
+    import torch
+    from sparse_attention_11_b200 import dsa
+    wl = prob.wl
+    T, H = wl.total_q, wl.heads
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    d_out = torch.randn((T, H, wl.dv), generator=gen, device="cuda").to(torch.bfloat16)
+    d_q = torch.empty((T, H, wl.dk), device="cuda")
+    d_kv = torch.zeros((wl.total_k, wl.dk), device="cuda")
+    ws = dsa.workspace(256)
+    run = lambda: dsa.dsa_sparse_attn_bwd(prob.seqs, prob.aa, prob.idx, wl.k, d_out, d_q, d_kv, d_kv[:, :wl.dv], ws)
+    for _ in range(warmup):
+        d_kv.zero_()
+        run()
+    st = torch.cuda.current_stream()
+    ts = []
+    for _ in range(steps):
+        d_kv.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        run()
+        e1.record(st)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    dsa.check_device_status(ws, "backward")
+    pos = np.concatenate([np.arange(sk - sq, sk) for sq, sk in zip(wl.seqlens_q, wl.seqlens_k)])
+    flops = 2.0 * H * (3 * wl.dk + 2 * wl.dv) * float(np.minimum(wl.k, pos + 1).sum())
+    ms = statistics.mean(ts)
+    return {"kernel": "attn_bwd_kernel (CUDA cores, fp32)", "ms": ms, "steps": steps,
+            "tflops": flops / (ms / 1e3) / 1e12, "flops_per_call": flops,
+            "tokens_per_s": T / (ms / 1e3)}
+
+
 def e2e_native(inp, prob, steps):
     """The same metric through the host-memory API, dsa_forward_host: every
     step copies its inputs from pinned host memory (the key-side tensors on the
@@ -534,6 +574,9 @@ def native(args):
         e2e_max = max_over_ranks(e2e_ms, ws_n, dev)
         res["e2e"] = {"value": ws_n * tokens_per_step / (e2e_max / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max, "api": "dsa_forward_host"}
+    # the backward runs on the fixed-k forward's selection, output and lse
+    if args.bwd and wl.attn_dtype == "bf16":
+        res["backward"] = backward_native(prob, max(1, min(args.steps, 3)), 1)
     # dynamic k last: it writes the problem's indices and output with another selection
     if not args.no_dynk and wl.name != "decode_b64":
         res["dynamic_k"] = dynamic_k_native(inp, prob, max(3, min(args.steps, 10)), args.warmup)

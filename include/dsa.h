@@ -139,7 +139,7 @@ typedef struct dsa_attn_args {
 DSA_API const char* dsa_status_string(int status);
 
 /* Library ABI version (major*1000 + minor).  1001: dsa_indexer_args gained
- * k_per_row. */
+ * k_per_row.  1002: dsa_sparse_attn_bwd. */
 DSA_API int dsa_version(void);
 
 /* Workspace bytes needed by `op` for this problem (k = top-k size, used by
@@ -187,6 +187,32 @@ DSA_API int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_score
  * DSA_ERR_INDEX. */
 DSA_API int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx,
                     int64_t ld_idx, int32_t k_sel, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Backward of dsa_sparse_attn (the training step's attention, §4.1 sparse
+ * stage; the attention itself §2.3, §3.1), over the same selection.
+ * aa describes the forward call: q, k, v, scale, dtype, heads, dk, dv and
+ * strides as for dsa_sparse_attn.  aa->out and aa->lse (required here) hold
+ * the forward's output and lse.  For every query t, head h and valid slot j
+ * of idx row t (row_j = cu_seqlens_k[b] + idx[t,j]):
+ *     P_j  = exp(scale * q[t,h].K[row_j] - lse[t,h])
+ *     dP_j = d_out[t,h] . V[row_j],   D = d_out[t,h] . out[t,h]
+ *     dS_j = P_j (dP_j - D)
+ *     d_q[t,h,:dk]      = scale * sum_j dS_j K[row_j,:dk]      (written)
+ *     d_k[row_j,:dk]   += scale * dS_j q[t,h,:dk]              (accumulated)
+ *     d_v[row_j,:dv]   += P_j d_out[t,h,:dv]                   (accumulated)
+ * d_out: same dtype as q, [total_q, heads, >= dv] with the given strides.
+ * d_q, d_k, d_v: float32.  d_k and d_v accumulate, so zero them first.
+ * d_v may be d_k itself (same pointer and stride): with V the first dv
+ * columns of K (MLA), d_k then receives the tied gradient.  Rows whose
+ * position is invalid are reported (DSA_ERR_INDEX) and their d_q is not
+ * written.  Supported: bf16 or f32, dk <= 576, dv <= 512, any head count.
+ * This first version runs on CUDA cores.  Workspace: a status header
+ * (256 bytes). */
+DSA_API int dsa_sparse_attn_bwd(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx,
+                                int32_t k_sel, const void* d_out, int64_t d_out_stride_tok,
+                                int64_t d_out_stride_head, float* d_q, int64_t d_q_stride_tok,
+                                int64_t d_q_stride_head, float* d_k, int64_t d_k_stride, float* d_v,
+                                int64_t d_v_stride, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /* Steps a1-a3 -- fold, then the indexer and the top-k: idx (int32
  * [total_q, ld_idx], ld_idx >= k) receives, for every query, its

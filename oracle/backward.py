@@ -62,7 +62,7 @@ def sparse_attn_fwd(q, K, V, idx, scale):
     return O, lse
 
 
-def sparse_attn_bwd(q, K, V, idx, scale, dO):
+def sparse_attn_bwd(q, K, V, idx, scale, dO, O=None):
     """Gradients of sum(dO * O) for sparse_attn_fwd.
 
     Returns dq [n,H,dk], dK [Nk,dk], dV [Nk,dv].  Every selected key
@@ -75,7 +75,11 @@ def sparse_attn_bwd(q, K, V, idx, scale, dO):
       dq   = scale * sum_j dz_j K[idx_j]
       dK[idx_j] += scale * dz_j q
       dV[idx_j] += P_j dO
-    Indices in a row must be distinct (a selection is a set)."""
+    Indices in a row must be distinct (a selection is a set).
+
+    O: optional forward output [n,H,dv].  When given, D = dO . O is taken
+    from it, as a training kernel does with the output it stored.  With the
+    exact output this is the same D."""
     q, K, V, dO = _f64(q), _f64(K), _f64(V), _f64(dO)
     n, H, dk = q.shape
     dq = np.zeros_like(q)
@@ -91,7 +95,10 @@ def sparse_attn_bwd(q, K, V, idx, scale, dO):
         P = np.exp(z - z.max(axis=1, keepdims=True))
         P /= P.sum(axis=1, keepdims=True)        # [H, m]
         dP = dO[t] @ V[sel].T                    # [H, m]
-        D = (P * dP).sum(axis=1, keepdims=True)
+        if O is None:
+            D = (P * dP).sum(axis=1, keepdims=True)
+        else:
+            D = (dO[t] * _f64(O[t])).sum(axis=1, keepdims=True)
         dz = P * (dP - D)
         dq[t] = scale * (dz @ K[sel])
         np.add.at(dK, sel, scale * (dz.T @ q[t]))

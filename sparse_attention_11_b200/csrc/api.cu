@@ -377,7 +377,7 @@ const char* dsa_status_string(int status) {
     return "unknown status";
 }
 
-int dsa_version(void) { return 1001; }
+int dsa_version(void) { return 1002; }
 
 int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexer_args* ia, const dsa_attn_args* aa,
                        size_t* bytes) {
@@ -447,6 +447,68 @@ int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_scores, int64
     r = check_ws(ws, ws_bytes, kHdr);
     if (r) return r;
     return run_topk(seqs, scores, ld_scores, row_begin, row_count, k, idx, ld_idx, hdr(ws), (cudaStream_t)stream);
+}
+
+int dsa_sparse_attn_bwd(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx,
+                        int32_t k_sel, const void* d_out, int64_t d_out_stride_tok, int64_t d_out_stride_head,
+                        float* d_q, int64_t d_q_stride_tok, int64_t d_q_stride_head, float* d_k, int64_t d_k_stride,
+                        float* d_v, int64_t d_v_stride, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (r) return r;
+    if (!aa) return DSA_ERR_INVALID_ARG;
+    if (aa->dtype != DSA_BF16 && aa->dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
+    if (aa->heads < 1 || aa->dk < 1 || aa->dv < 1) return DSA_ERR_INVALID_ARG;
+    if (aa->dk > kBwdMaxDk || aa->dv > kBwdMaxDv || aa->heads > 65535 * 16) return DSA_ERR_UNSUPPORTED;
+    if (k_sel < 0 || ld_idx < k_sel) return DSA_ERR_INVALID_ARG;
+    if (seqs->total_q && (!aa->q || !aa->out || !aa->lse || !d_out || !d_q || (k_sel && !idx)))
+        return DSA_ERR_INVALID_ARG;
+    if (seqs->total_k && (!aa->k || !aa->v || !d_k || !d_v)) return DSA_ERR_INVALID_ARG;
+    if (aa->q_stride_head < aa->dk || aa->q_stride_tok < (int64_t)aa->heads * aa->q_stride_head) return DSA_ERR_INVALID_ARG;
+    if (aa->out_stride_head < aa->dv || aa->out_stride_tok < (int64_t)aa->heads * aa->out_stride_head)
+        return DSA_ERR_INVALID_ARG;
+    if (d_out_stride_head < aa->dv || d_out_stride_tok < (int64_t)aa->heads * d_out_stride_head)
+        return DSA_ERR_INVALID_ARG;
+    if (d_q_stride_head < aa->dk || d_q_stride_tok < (int64_t)aa->heads * d_q_stride_head) return DSA_ERR_INVALID_ARG;
+    if (aa->k_stride < aa->dk || aa->v_stride < aa->dv || d_k_stride < aa->dk || d_v_stride < aa->dv)
+        return DSA_ERR_INVALID_ARG;
+    r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    if (seqs->total_q == 0) return DSA_OK;
+    AttnBwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.sv = seq_view(seqs);
+    a.total_q = seqs->total_q;
+    a.heads = aa->heads;
+    a.dk = aa->dk;
+    a.dv = aa->dv;
+    a.scale = aa->scale;
+    a.q = aa->q;
+    a.q_stride_tok = aa->q_stride_tok;
+    a.q_stride_head = aa->q_stride_head;
+    a.k = aa->k;
+    a.k_stride = aa->k_stride;
+    a.v = aa->v;
+    a.v_stride = aa->v_stride;
+    a.out = aa->out;
+    a.out_stride_tok = aa->out_stride_tok;
+    a.out_stride_head = aa->out_stride_head;
+    a.lse = aa->lse;
+    a.dout = d_out;
+    a.dout_stride_tok = d_out_stride_tok;
+    a.dout_stride_head = d_out_stride_head;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.k_sel = k_sel;
+    a.d_q = d_q;
+    a.d_q_stride_tok = d_q_stride_tok;
+    a.d_q_stride_head = d_q_stride_head;
+    a.d_k = d_k;
+    a.d_k_stride = d_k_stride;
+    a.d_v = d_v;
+    a.d_v_stride = d_v_stride;
+    a.st = hdr(ws);
+    if (!launch_attn_bwd(a, aa->dtype == DSA_BF16, (cudaStream_t)stream)) return DSA_ERR_CUDA;
+    return cuda_status();
 }
 
 int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel,

@@ -127,4 +127,37 @@ struct AttnTcArgs {
 };
 bool launch_attn_tc(const AttnTcArgs& a, cudaStream_t s);
 
+// ---------------------------------------------------------------------------
+// Backward of the sparse attention (CUDA cores, fp32 arithmetic).
+// ---------------------------------------------------------------------------
+constexpr int kBwdMaxDk = 576, kBwdMaxDv = 512;
+struct AttnBwdArgs {
+    SeqView sv;
+    int64_t total_q;
+    int heads, dk, dv;
+    float scale;
+    const void* q;          // [total_q, heads, >= dk] (bf16 or f32)
+    int64_t q_stride_tok, q_stride_head;
+    const void* k;          // K rows, row stride k_stride
+    int64_t k_stride;
+    const void* v;          // V rows, row stride v_stride (may alias k)
+    int64_t v_stride;
+    const void* out;        // the forward's output
+    int64_t out_stride_tok, out_stride_head;
+    const float* lse;       // the forward's lse, [total_q, heads]
+    const void* dout;       // gradient of the output
+    int64_t dout_stride_tok, dout_stride_head;
+    const int32_t* idx;
+    int64_t ld_idx;
+    int k_sel;
+    float* d_q;             // written
+    int64_t d_q_stride_tok, d_q_stride_head;
+    float* d_k;             // accumulated
+    int64_t d_k_stride;
+    float* d_v;             // accumulated (may alias d_k)
+    int64_t d_v_stride;
+    StatusHdr* st;
+};
+bool launch_attn_bwd(const AttnBwdArgs& a, int dtype_bf16, cudaStream_t s);
+
 }  // namespace dsa

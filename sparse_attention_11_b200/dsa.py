@@ -49,20 +49,24 @@ _lib.dsa_fold.argtypes = [_S, _IA, _P, _P, _P, _SZ, _P]
 _lib.dsa_index_scores.argtypes = [_S, _IA, _I64, _I64, _P, _I64, _P, _SZ, _P]
 _lib.dsa_topk.argtypes = [_S, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_sparse_attn.argtypes = [_S, _AA, _P, _I64, _I32, _P, _SZ, _P]
+_lib.dsa_sparse_attn_bwd.argtypes = [_S, _AA, _P, _I64, _I32, _P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _I64,
+                                     _P, _SZ, _P]
 _lib.dsa_forward.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_forward_host.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P, _P, _P]
 _lib.dsa_select.argtypes = [_S, _IA, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_select_noalloc.argtypes = [_S, _IA, _I32, _P, _I64, _P]
 _lib.dsa_sync_status.argtypes = [_P, _P, ctypes.POINTER(_I64)]
 _lib.dsa_selftest_wait_timeout.argtypes = [_P, _SZ, _I64, _P]
-for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_sparse_attn_bwd",
+           "dsa_forward",
            "dsa_forward_host",
            "dsa_select", "dsa_select_noalloc",
            "dsa_sync_status", "dsa_selftest_wait_timeout"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk",
-            "dsa_sparse_attn", "dsa_forward", "dsa_forward_host", "dsa_select", "dsa_select_noalloc", "dsa_sync_status",
+            "dsa_sparse_attn", "dsa_sparse_attn_bwd", "dsa_forward", "dsa_forward_host", "dsa_select",
+            "dsa_select_noalloc", "dsa_sync_status",
             "dsa_selftest_wait_timeout")
 
 
@@ -177,6 +181,18 @@ def dsa_topk(seqs, scores, row_begin, row_count, k, idx, ws):
 def dsa_sparse_attn(seqs, aa, idx, k_sel, ws):
     _check(_lib.dsa_sparse_attn(ctypes.byref(seqs.c), ctypes.byref(aa), _ptr(idx), idx.stride(0), k_sel, _ptr(ws),
                                 ws.numel(), _stream()), "dsa_sparse_attn")
+
+
+def dsa_sparse_attn_bwd(seqs, aa, idx, k_sel, d_out, d_q, d_k, d_v, ws):
+    """Backward of dsa_sparse_attn.  aa is the forward's attn_args (its out
+    and lse hold the forward's results; lse is required).  d_out [T,H,dv]
+    has q's dtype; d_q [T,H,dk] float32 is written; d_k [Tk,>=dk] and d_v
+    [Tk,>=dv] float32 accumulate (zero them first; d_v may be a view of d_k's
+    first dv columns for the MLA-tied gradient)."""
+    _check(_lib.dsa_sparse_attn_bwd(ctypes.byref(seqs.c), ctypes.byref(aa), _ptr(idx), idx.stride(0), k_sel,
+                                    _ptr(d_out), d_out.stride(0), d_out.stride(1), _ptr(d_q), d_q.stride(0),
+                                    d_q.stride(1), _ptr(d_k), d_k.stride(0), _ptr(d_v), d_v.stride(0), _ptr(ws),
+                                    ws.numel(), _stream()), "dsa_sparse_attn_bwd")
 
 
 def dsa_forward_host(seqs, ia, aa, k, idx_out, ws, h2d_stream=None, d2h_stream=None):

@@ -133,6 +133,33 @@ def test_selection_path_workspace(lib):
         assert size(b, tq, tk, mq, mk) < tq * k * 4 + tq * 256 + (1 << 20), (b, tq, tk)
 
 
+def test_backward_validation(lib):
+    """dsa_sparse_attn_bwd rejects bad arguments before launching: a missing
+    lse or gradient buffer, unsupported dtype or dims, short strides, a short
+    workspace."""
+    S = _fake_seqs(lib, tq=64, tk=64)
+    P = ctypes.c_void_p
+    h, dk, dv = 128, 576, 512
+
+    def aa(dtype=lib.DSA_BF16, dk_=dk, dv_=dv, lse=0x500000):
+        return lib.dsa_attn_args(dtype, h, dk_, dv_, 0x100000, h * dk_, dk_, 0x200000, dk_, 0x200000, dk_, 0.1,
+                                 0x400000, h * dv_, dv_, lse)
+
+    def call(a, d_out=0x600000, dq=0x700000, dk_=0x800000, dks=dk, dvs=dk, dos=(h * dv, dv), ws_bytes=1 << 20):
+        return lib.raw_call("dsa_sparse_attn_bwd", ctypes.byref(S), ctypes.byref(a), P(0x900000), 64, 64, P(d_out),
+                            dos[0], dos[1], P(dq), h * dk, dk, P(dk_), dks, P(dk_), dvs, P(0x10000), ws_bytes, None)
+
+    assert call(aa(lse=None)) == lib.DSA_ERR_INVALID_ARG
+    assert call(aa(), d_out=0) == lib.DSA_ERR_INVALID_ARG
+    assert call(aa(), dq=0) == lib.DSA_ERR_INVALID_ARG
+    assert call(aa(), dk_=0) == lib.DSA_ERR_INVALID_ARG
+    assert call(aa(lib.DSA_E4M3)) == lib.DSA_ERR_UNSUPPORTED
+    assert call(aa(dk_=640)) == lib.DSA_ERR_UNSUPPORTED
+    assert call(aa(), dks=500) == lib.DSA_ERR_INVALID_ARG
+    assert call(aa(), dos=(h * dv, 100)) == lib.DSA_ERR_INVALID_ARG
+    assert call(aa(), ws_bytes=64) == lib.DSA_ERR_WORKSPACE
+
+
 def test_forward_host_validation(lib):
     """The host-memory forward rejects non-packed or fp32 attention operands
     and short workspaces before touching the device; its workspace holds the

@@ -66,6 +66,20 @@ def test_attention_backward_finite_differences():
     assert np.all(dK[unused] == 0) and np.all(dV[unused] == 0)
 
 
+def test_attention_backward_stored_output():
+    """D from the stored output equals D = sum_j P_j dP_j when the output is
+    exact; a perturbed output moves only D."""
+    q, K, V, idx, dO, sc = _attn_case(seed=10)
+    O, _ = B.sparse_attn_fwd(q, K, V, idx, sc)
+    a = B.sparse_attn_bwd(q, K, V, idx, sc, dO)
+    b = B.sparse_attn_bwd(q, K, V, idx, sc, dO, O=O)
+    for x, y in zip(a, b):
+        assert np.allclose(x, y, rtol=0, atol=1e-13)
+    c = B.sparse_attn_bwd(q, K, V, idx, sc, dO, O=O * 1.01)
+    assert np.array_equal(c[2], a[2])           # dV does not involve D
+    assert not np.allclose(c[0], a[0])          # dq does
+
+
 def test_attention_backward_single_key():
     q, K, V, idx, dO, sc = _attn_case(seed=1)
     idx[:, 1:] = -1
