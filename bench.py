@@ -374,14 +374,16 @@ def context_parallel_native(args, ws_n, rank, dev, sampler):
     lse = torch.empty((n, wl.heads), dtype=torch.float32, device=dev)
     idx = torch.empty((n, wl.k), dtype=torch.int32, device=dev)
     st = torch.cuda.current_stream()
+    run = cp.ContextParallelForward(plans, rank, wl.k, q_idx, q_sc, W_index, q, wl.dk, wl.dv, wl.scale, out, lse,
+                                    idx, k_idx_sh.dtype, kv_sh.dtype)
 
     def step():
-        cp.forward(plans, rank, wl.k, q_idx, q_sc, W_index, k_idx_sh, k_sc_sh, q, kv_sh, wl.dv, wl.scale, out, lse,
-                   idx)
+        run.step(k_idx_sh, k_sc_sh, kv_sh)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    run.check("context-parallel warm-up")
     barrier(ws_n)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -393,6 +395,7 @@ def context_parallel_native(args, ws_n, rank, dev, sampler):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     barrier(ws_n)
+    run.check("context-parallel timed steps")
     ms_max = max_over_ranks(t0.elapsed_time(t1), ws_n, dev)
     return {
         "metric": METRIC, "value": L * args.steps / (ms_max / 1e3), "unit": "tokens/s", "n_gpus": ws_n,

@@ -107,9 +107,10 @@ def chunk_seqs(chunk, device):
     return dsa.Seqs([0, b - a], [0, b], device=device)
 
 
-def all_gather_rows(x, plans, rank, group=None):
+def all_gather_rows(x, plans, rank, group=None, out=None):
     """Assemble the full [L, ...] tensor from every rank's shard `x` (the rows
-    of plans[rank], in chunk order).
+    of plans[rank], in chunk order), into `out` when given (rows in sequence
+    order; it must be [L, ...] of x's dtype), else into a new tensor.
 
     One all-gather per chunk slot (the j-th chunk of every rank).  Each
     rank's piece is padded to the slot's longest chunk, because the
@@ -120,7 +121,12 @@ def all_gather_rows(x, plans, rank, group=None):
 
     world = len(plans)
     L = max(e for p in plans for _, e in p) if any(plans) else 0
-    full = torch.empty((L,) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+    if out is not None:
+        if tuple(out.shape) != (L,) + tuple(x.shape[1:]) or out.dtype != x.dtype:
+            raise ValueError("out must be [L, ...] with the shard's dtype")
+        full = out
+    else:
+        full = torch.empty((L,) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
     if world == 1:
         off = 0
         for s, e in plans[0]:
@@ -187,13 +193,47 @@ class LocalForward:
         dsa.check_device_status(self.ws, where)
 
 
+class ContextParallelForward:
+    """One rank's context-parallel forward, with every buffer allocated once:
+    the gathered key side (index codes, their scales, the KV rows) and the
+    per-chunk calls of LocalForward over them.  Each step all-gathers the
+    ranks' key-side shards into those buffers and runs the rank's chunks.
+
+    q_idx, q_scale, q, out, lse, idx: this rank's rows in chunk order, as in
+    LocalForward.  The shards passed to step() are this rank's key-side rows
+    in chunk order: k_idx [n, 128], k_scale [n] or None, kv [n, dk].  V is
+    the first dv columns of the gathered KV rows (MLA)."""
+
+    def __init__(self, plans, rank, k, q_idx, q_scale, W, q, dk, dv, scale, out, lse, idx, k_idx_dtype,
+                 kv_dtype, group=None):
+        self.plans, self.rank, self.group = plans, rank, group
+        L = max(e for p in plans for _, e in p)
+        dev = q.device
+        self.k_idx = torch.empty((L, 128), dtype=k_idx_dtype, device=dev)
+        self.k_scale = torch.empty((L,), dtype=torch.float32, device=dev) if q_scale is not None else None
+        self.kv = torch.empty((L, dk), dtype=kv_dtype, device=dev)
+        self.local = LocalForward(plans[rank], k, q_idx, q_scale, W, self.k_idx, self.k_scale, q, self.kv,
+                                  self.kv[:, :dv], scale, out, lse, idx)
+
+    def step(self, k_idx_shard, k_scale_shard, kv_shard):
+        all_gather_rows(k_idx_shard, self.plans, self.rank, self.group, out=self.k_idx)
+        if self.k_scale is not None:
+            all_gather_rows(k_scale_shard, self.plans, self.rank, self.group, out=self.k_scale)
+        all_gather_rows(kv_shard, self.plans, self.rank, self.group, out=self.kv)
+        self.local()
+
+    def check(self, where="context-parallel forward"):
+        self.local.check(where)
+
+
 def forward(plans, rank, k, q_idx, q_scale, W, k_idx_shard, k_scale_shard, q, kv_shard, dv, scale, out, lse, idx,
             v_shard=None, group=None):
-    """Context-parallel forward on this rank: all-gather the key side
-    (indexer codes, their scales, the KV rows), then run the rank's chunks.
-    V is the first dv columns of the KV rows (the MLA latent part) unless
-    v_shard gives V's rows separately.  Returns the gathered
-    (k_idx, k_scale, K, V) for reuse."""
+    """Context-parallel forward on this rank in one call: all-gather the key
+    side (indexer codes, their scales, the KV rows), then run the rank's
+    chunks.  V is the first dv columns of the KV rows (the MLA latent part)
+    unless v_shard gives V's rows separately.  Returns the gathered
+    (k_idx, k_scale, K, V).  Repeated steps should use
+    ContextParallelForward, which allocates once."""
     k_idx = all_gather_rows(k_idx_shard, plans, rank, group)
     k_scale = all_gather_rows(k_scale_shard, plans, rank, group) if k_scale_shard is not None else None
     K = all_gather_rows(kv_shard, plans, rank, group)

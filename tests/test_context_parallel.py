@@ -110,6 +110,11 @@ def _worker(rank, world, port, scheme, q):
         ok_types = (np.array_equal(cpm.all_gather_rows(torch.from_numpy(codes[rows]), p, rank).numpy(), codes) and
                     np.array_equal(cpm.all_gather_rows(torch.from_numpy(scales[rows]), p, rank).numpy(), scales) and
                     torch.equal(cpm.all_gather_rows(kv[torch.from_numpy(rows)], p, rank), kv))
+        # into a preallocated buffer (the per-step form), twice over the same buffer
+        buf = torch.full_like(kv, float("nan"))
+        for _ in range(2):
+            got = cpm.all_gather_rows(kv[torch.from_numpy(rows)], p, rank, out=buf)
+            ok_types = ok_types and got is buf and torch.equal(buf, kv)
         # this rank's rows at the chunk positions, against the gathered keys
         pos = np.concatenate([np.arange(a, b) for a, b in mine]).astype(np.int64)
         kb = np.zeros_like(pos)
