@@ -188,3 +188,25 @@ def test_forward_host_validation(lib):
     f32 = lib.dsa_attn_args(lib.DSA_F32, 4, 64, 64, 0x100000, 256, 64, 0x200000, 64, 0x300000, 64, 0.1,
                             0x400000, 256, 64, None)
     assert call(f32, 1 << 40) == lib.DSA_ERR_UNSUPPORTED
+
+
+def test_bench_launch_count_follows_library_path(lib):
+    """bench.py counts 4 launches per prefill step where the library selects
+    in two launches, else 3.  The library's choice shows in its workspace:
+    only the two-launch (and scan) paths hold a score buffer."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_attention_11_b200 import workloads as W
+    n = ctypes.c_size_t(0)
+    ia = lib.dsa_indexer_args(lib.DSA_E4M3, 0x100000, 0x110000, lib.DSA_BF16, 0x200000, 0x300000, 0x310000)
+    shapes = [((8192,), (8192,)), ((32768,), (32768,)), ((2048,), (2048,)), ((3000,), (3000,)),
+              ((18944,), (18944,)), ((18816,), (18816,)), ((700, 1500, 129), (700, 1500, 129)),
+              ((2048,), (32768,))]
+    for sq, sk in shapes:
+        wl = W.custom("probe", sq, sk, base="prefill_l8192")
+        S = lib.dsa_seqs(len(sq), sum(sq), sum(sk), max(sq), max(sk), 0x1000, 0x2000)
+        assert lib.raw_call("dsa_workspace_size", lib.DSA_OP_FORWARD, ctypes.byref(S), wl.k, ctypes.byref(ia), None,
+                            ctypes.byref(n)) == 0
+        has_scores = n.value >= sum(sq) * max(sk) * 4 + sum(sq) * wl.k * 4  # score buffer on top of the index rows
+        assert bench.step_launches(wl) == (4 if has_scores else 3), (sq, sk, n.value)
