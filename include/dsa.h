@@ -139,7 +139,8 @@ typedef struct dsa_attn_args {
 DSA_API const char* dsa_status_string(int status);
 
 /* Library ABI version (major*1000 + minor).  1001: dsa_indexer_args gained
- * k_per_row.  1002: dsa_sparse_attn_bwd. */
+ * k_per_row.  1002: dsa_sparse_attn_bwd.  1003: dsa_attn_target,
+ * dsa_indexer_kl. */
 DSA_API int dsa_version(void);
 
 /* Workspace bytes needed by `op` for this problem (k = top-k size, used by
@@ -213,6 +214,38 @@ DSA_API int dsa_sparse_attn_bwd(const dsa_seqs* seqs, const dsa_attn_args* aa, c
                                 int64_t d_out_stride_head, float* d_q, int64_t d_q_stride_tok,
                                 int64_t d_q_stride_head, float* d_k, int64_t d_k_stride, float* d_v,
                                 int64_t d_v_stride, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Training target of the indexer's KL distillation in the sparse stage
+ * (§4.1): the main attention's probabilities of every selected key, averaged
+ * over the heads,
+ *     p[t, j] = (1/heads) sum_h exp(scale * q[t,h].K[row_j] - lse[t,h])
+ * for every valid slot j of idx row t, and 0 for empty slots.  aa describes
+ * the forward call (q, k, scale, dtype, heads, dk; aa->lse, required, holds
+ * the forward's lse; v and out are not read).  p: float [total_q, ld_p],
+ * ld_p >= k_sel.  The call zeroes the whole array, then writes it.  Over a
+ * row's valid slots, p sums to 1.  Supported: bf16 or f32, dk <= 576.
+ * Workspace: a status header (256 bytes). */
+DSA_API int dsa_attn_target(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx,
+                            int32_t k_sel, float* p, int64_t ld_p, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* The indexer's KL distillation loss over the selection and its gradients
+ * (§4.1, sparse stage; I from §2.2).  Real-valued fp32 inputs: the indexer
+ * query q_idx [total_q, q_stride >= 128], W [128,128] row-major
+ * (u = q W), and the indexer keys k_idx [total_k, k_stride >= 128].  For
+ * every query t over the valid slots j of its idx row:
+ *     x_j = (q_t W) . k_j,  I_j = max(x_j, 0),  r = softmax_j(I)
+ *     loss[t] = sum_j p_j (log p_j - log r_j)    (terms with p_j = 0 drop)
+ *     G_j = (r_j - p_j) [x_j > 0]
+ *     d_q[t] = W sum_j G_j k_j                          (written)
+ *     d_W   += q_t^T sum_j G_j k_j                      (accumulated)
+ *     d_k[row_j] += G_j (q_t W)                         (accumulated)
+ * p is the target per slot (e.g. from dsa_attn_target), summing to 1 over
+ * each row's valid slots.  loss (float [total_q]) may be NULL.  Zero d_W and
+ * d_k first.  k_sel <= 16384.  Workspace: a status header (256 bytes). */
+DSA_API int dsa_indexer_kl(const dsa_seqs* seqs, const float* q_idx, int64_t q_stride, const float* W,
+                           const float* k_idx, int64_t k_stride, const int32_t* idx, int64_t ld_idx, int32_t k_sel,
+                           const float* p, int64_t ld_p, float* loss, float* d_q, int64_t d_q_stride, float* d_W,
+                           float* d_k, int64_t d_k_stride, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /* Steps a1-a3 -- fold, then the indexer and the top-k: idx (int32
  * [total_q, ld_idx], ld_idx >= k) receives, for every query, its

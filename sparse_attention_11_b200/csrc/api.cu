@@ -377,7 +377,7 @@ const char* dsa_status_string(int status) {
     return "unknown status";
 }
 
-int dsa_version(void) { return 1002; }
+int dsa_version(void) { return 1003; }
 
 int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexer_args* ia, const dsa_attn_args* aa,
                        size_t* bytes) {
@@ -508,6 +508,87 @@ int dsa_sparse_attn_bwd(const dsa_seqs* seqs, const dsa_attn_args* aa, const int
     a.d_v_stride = d_v_stride;
     a.st = hdr(ws);
     if (!launch_attn_bwd(a, aa->dtype == DSA_BF16, (cudaStream_t)stream)) return DSA_ERR_CUDA;
+    return cuda_status();
+}
+
+int dsa_attn_target(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel,
+                    float* p, int64_t ld_p, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (r) return r;
+    if (!aa) return DSA_ERR_INVALID_ARG;
+    if (aa->dtype != DSA_BF16 && aa->dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
+    if (aa->heads < 1 || aa->dk < 1) return DSA_ERR_INVALID_ARG;
+    if (aa->dk > kBwdMaxDk || aa->heads > 65535 * 16) return DSA_ERR_UNSUPPORTED;
+    if (k_sel < 0 || ld_idx < k_sel || ld_p < k_sel) return DSA_ERR_INVALID_ARG;
+    if (seqs->total_q && (!aa->q || !aa->lse || !p || (k_sel && !idx))) return DSA_ERR_INVALID_ARG;
+    if (seqs->total_k && !aa->k) return DSA_ERR_INVALID_ARG;
+    if (aa->q_stride_head < aa->dk || aa->q_stride_tok < (int64_t)aa->heads * aa->q_stride_head) return DSA_ERR_INVALID_ARG;
+    if (aa->k_stride < aa->dk) return DSA_ERR_INVALID_ARG;
+    r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    if (seqs->total_q == 0) return DSA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(p, 0, (size_t)seqs->total_q * (size_t)ld_p * sizeof(float), st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    AttnPmeanArgs a;
+    memset(&a, 0, sizeof(a));
+    a.sv = seq_view(seqs);
+    a.total_q = seqs->total_q;
+    a.heads = aa->heads;
+    a.dk = aa->dk;
+    a.scale = aa->scale;
+    a.q = aa->q;
+    a.q_stride_tok = aa->q_stride_tok;
+    a.q_stride_head = aa->q_stride_head;
+    a.k = aa->k;
+    a.k_stride = aa->k_stride;
+    a.lse = aa->lse;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.k_sel = k_sel;
+    a.p = p;
+    a.ld_p = ld_p;
+    a.st = hdr(ws);
+    if (!launch_attn_pmean(a, aa->dtype == DSA_BF16, st)) return DSA_ERR_CUDA;
+    return cuda_status();
+}
+
+int dsa_indexer_kl(const dsa_seqs* seqs, const float* q_idx, int64_t q_stride, const float* W, const float* k_idx,
+                   int64_t k_stride, const int32_t* idx, int64_t ld_idx, int32_t k_sel, const float* p, int64_t ld_p,
+                   float* loss, float* d_q, int64_t d_q_stride, float* d_W, float* d_k, int64_t d_k_stride, void* ws,
+                   size_t ws_bytes, dsa_stream_t stream) {
+    int r = check_seqs(seqs);
+    if (r) return r;
+    if (k_sel < 0 || k_sel > 16384 || ld_idx < k_sel || ld_p < k_sel) return DSA_ERR_INVALID_ARG;
+    if (!W || !d_W) return DSA_ERR_INVALID_ARG;
+    if (seqs->total_q && (!q_idx || !p || !d_q || (k_sel && !idx))) return DSA_ERR_INVALID_ARG;
+    if (seqs->total_k && (!k_idx || !d_k)) return DSA_ERR_INVALID_ARG;
+    if (q_stride < 128 || k_stride < 128 || d_q_stride < 128 || d_k_stride < 128) return DSA_ERR_INVALID_ARG;
+    r = check_ws(ws, ws_bytes, kHdr);
+    if (r) return r;
+    if (seqs->total_q == 0) return DSA_OK;
+    IndexerKlArgs a;
+    memset(&a, 0, sizeof(a));
+    a.sv = seq_view(seqs);
+    a.total_q = seqs->total_q;
+    a.q = q_idx;
+    a.q_stride = q_stride;
+    a.W = W;
+    a.k = k_idx;
+    a.k_stride = k_stride;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.k_sel = k_sel;
+    a.p = p;
+    a.ld_p = ld_p;
+    a.loss = loss;
+    a.d_q = d_q;
+    a.d_q_stride = d_q_stride;
+    a.d_W = d_W;
+    a.d_k = d_k;
+    a.d_k_stride = d_k_stride;
+    a.st = hdr(ws);
+    if (!launch_indexer_kl(a, (cudaStream_t)stream)) return DSA_ERR_CUDA;
     return cuda_status();
 }
 

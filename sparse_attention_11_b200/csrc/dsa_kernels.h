@@ -160,4 +160,50 @@ struct AttnBwdArgs {
 };
 bool launch_attn_bwd(const AttnBwdArgs& a, int dtype_bf16, cudaStream_t s);
 
+// ---------------------------------------------------------------------------
+// Indexer KL distillation (sparse stage): the attention target over the
+// selected rows, then the KL loss and its gradients (CUDA cores, fp32).
+// ---------------------------------------------------------------------------
+struct AttnPmeanArgs {
+    SeqView sv;
+    int64_t total_q;
+    int heads, dk;
+    float scale;
+    const void* q;          // [total_q, heads, >= dk]
+    int64_t q_stride_tok, q_stride_head;
+    const void* k;          // K rows, row stride k_stride
+    int64_t k_stride;
+    const float* lse;       // the forward's lse, [total_q, heads]
+    const int32_t* idx;
+    int64_t ld_idx;
+    int k_sel;
+    float* p;               // [total_q, ld_p], accumulated over head groups (zeroed by the caller)
+    int64_t ld_p;
+    StatusHdr* st;
+};
+bool launch_attn_pmean(const AttnPmeanArgs& a, int dtype_bf16, cudaStream_t s);
+
+struct IndexerKlArgs {
+    SeqView sv;
+    int64_t total_q;
+    const float* q;         // [total_q, 128] real-valued indexer query
+    int64_t q_stride;
+    const float* W;         // [128, 128], u = q W
+    const float* k;         // [total_k, 128] real-valued indexer keys
+    int64_t k_stride;
+    const int32_t* idx;
+    int64_t ld_idx;
+    int k_sel;
+    const float* p;         // target per slot [total_q, ld_p]
+    int64_t ld_p;
+    float* loss;            // [total_q] per query (nullable)
+    float* d_q;             // [total_q, d_q_stride], written
+    int64_t d_q_stride;
+    float* d_W;             // [128, 128], accumulated
+    float* d_k;             // [total_k, d_k_stride], accumulated
+    int64_t d_k_stride;
+    StatusHdr* st;
+};
+bool launch_indexer_kl(const IndexerKlArgs& a, cudaStream_t s);
+
 }  // namespace dsa

@@ -49,6 +49,9 @@ _lib.dsa_fold.argtypes = [_S, _IA, _P, _P, _P, _SZ, _P]
 _lib.dsa_index_scores.argtypes = [_S, _IA, _I64, _I64, _P, _I64, _P, _SZ, _P]
 _lib.dsa_topk.argtypes = [_S, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ, _P]
 _lib.dsa_sparse_attn.argtypes = [_S, _AA, _P, _I64, _I32, _P, _SZ, _P]
+_lib.dsa_attn_target.argtypes = [_S, _AA, _P, _I64, _I32, _P, _I64, _P, _SZ, _P]
+_lib.dsa_indexer_kl.argtypes = [_S, _P, _I64, _P, _P, _I64, _P, _I64, _I32, _P, _I64, _P, _P, _I64, _P, _P, _I64, _P,
+                                _SZ, _P]
 _lib.dsa_sparse_attn_bwd.argtypes = [_S, _AA, _P, _I64, _I32, _P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _I64,
                                      _P, _SZ, _P]
 _lib.dsa_forward.argtypes = [_S, _IA, _AA, _I32, _P, _I64, _P, _SZ, _P]
@@ -58,6 +61,7 @@ _lib.dsa_select_noalloc.argtypes = [_S, _IA, _I32, _P, _I64, _P]
 _lib.dsa_sync_status.argtypes = [_P, _P, ctypes.POINTER(_I64)]
 _lib.dsa_selftest_wait_timeout.argtypes = [_P, _SZ, _I64, _P]
 for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_sparse_attn_bwd",
+           "dsa_attn_target", "dsa_indexer_kl",
            "dsa_forward",
            "dsa_forward_host",
            "dsa_select", "dsa_select_noalloc",
@@ -65,7 +69,8 @@ for _f in ("dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk", "ds
     getattr(_lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_fold", "dsa_index_scores", "dsa_topk",
-            "dsa_sparse_attn", "dsa_sparse_attn_bwd", "dsa_forward", "dsa_forward_host", "dsa_select",
+            "dsa_sparse_attn", "dsa_sparse_attn_bwd", "dsa_attn_target", "dsa_indexer_kl", "dsa_forward",
+            "dsa_forward_host", "dsa_select",
             "dsa_select_noalloc", "dsa_sync_status",
             "dsa_selftest_wait_timeout")
 
@@ -193,6 +198,24 @@ def dsa_sparse_attn_bwd(seqs, aa, idx, k_sel, d_out, d_q, d_k, d_v, ws):
                                     _ptr(d_out), d_out.stride(0), d_out.stride(1), _ptr(d_q), d_q.stride(0),
                                     d_q.stride(1), _ptr(d_k), d_k.stride(0), _ptr(d_v), d_v.stride(0), _ptr(ws),
                                     ws.numel(), _stream()), "dsa_sparse_attn_bwd")
+
+
+def dsa_attn_target(seqs, aa, idx, k_sel, p, ws):
+    """Head-averaged attention probabilities of the selected keys (the
+    indexer's KL target).  aa is the forward's attn_args (lse required);
+    p float32 [T, >= k_sel] is zeroed and written."""
+    _check(_lib.dsa_attn_target(ctypes.byref(seqs.c), ctypes.byref(aa), _ptr(idx), idx.stride(0), k_sel, _ptr(p),
+                                p.stride(0), _ptr(ws), ws.numel(), _stream()), "dsa_attn_target")
+
+
+def dsa_indexer_kl(seqs, q_idx, W, k_idx, idx, k_sel, p, loss, d_q, d_W, d_k, ws):
+    """The indexer's KL loss over the selection and its gradients (float32
+    tensors: q_idx [T,128], W [128,128], k_idx [Tk,128], p [T,>=k_sel];
+    loss [T] or None; d_q written; d_W, d_k accumulated)."""
+    _check(_lib.dsa_indexer_kl(ctypes.byref(seqs.c), _ptr(q_idx), q_idx.stride(0), _ptr(W), _ptr(k_idx),
+                               k_idx.stride(0), _ptr(idx), idx.stride(0), k_sel, _ptr(p), p.stride(0), _ptr(loss),
+                               _ptr(d_q), d_q.stride(0), _ptr(d_W), _ptr(d_k), d_k.stride(0), _ptr(ws), ws.numel(),
+                               _stream()), "dsa_indexer_kl")
 
 
 def dsa_forward_host(seqs, ia, aa, k, idx_out, ws, h2d_stream=None, d2h_stream=None):

@@ -160,6 +160,35 @@ def test_backward_validation(lib):
     assert call(aa(), ws_bytes=64) == lib.DSA_ERR_WORKSPACE
 
 
+def test_kl_entry_points_validation(lib):
+    """dsa_attn_target and dsa_indexer_kl reject bad arguments before
+    launching anything."""
+    S = _fake_seqs(lib, tq=64, tk=64)
+    P = ctypes.c_void_p
+    h, dk, dv = 128, 576, 512
+    ok_aa = lib.dsa_attn_args(lib.DSA_BF16, h, dk, dv, 0x100000, h * dk, dk, 0x200000, dk, 0x200000, dk, 0.1,
+                              0x400000, h * dv, dv, 0x500000)
+    no_lse = lib.dsa_attn_args(lib.DSA_BF16, h, dk, dv, 0x100000, h * dk, dk, 0x200000, dk, 0x200000, dk, 0.1,
+                               0x400000, h * dv, dv, None)
+    tgt = lambda a, ldp=64, ws_bytes=1 << 20: lib.raw_call("dsa_attn_target", ctypes.byref(S), ctypes.byref(a),
+                                                           P(0x900000), 64, 64, P(0xA00000), ldp, P(0x10000),
+                                                           ws_bytes, None)
+    assert tgt(no_lse) == lib.DSA_ERR_INVALID_ARG
+    assert tgt(ok_aa, ldp=32) == lib.DSA_ERR_INVALID_ARG
+    assert tgt(ok_aa, ws_bytes=64) == lib.DSA_ERR_WORKSPACE
+
+    def kl(q=0x100000, qs=128, W=0x200000, k_sel=64, p=0xA00000, ws_bytes=1 << 20):
+        return lib.raw_call("dsa_indexer_kl", ctypes.byref(S), P(q), qs, P(W), P(0x300000), 128, P(0x900000), 64,
+                            k_sel, P(p), 64, None, P(0x700000), 128, P(0x800000), P(0x600000), 128, P(0x10000),
+                            ws_bytes, None)
+    assert kl(q=0) == lib.DSA_ERR_INVALID_ARG
+    assert kl(qs=64) == lib.DSA_ERR_INVALID_ARG
+    assert kl(W=0) == lib.DSA_ERR_INVALID_ARG
+    assert kl(p=0) == lib.DSA_ERR_INVALID_ARG
+    assert kl(k_sel=100) == lib.DSA_ERR_INVALID_ARG  # ld_idx 64 < k_sel
+    assert kl(ws_bytes=64) == lib.DSA_ERR_WORKSPACE
+
+
 def test_forward_host_validation(lib):
     """The host-memory forward rejects non-packed or fp32 attention operands
     and short workspaces before touching the device; its workspace holds the
