@@ -179,6 +179,22 @@ def workload_info(wl):
     return {"tokens": int(wl.total_q), "sum_sel": int(sel.sum()), "pairs": int((pos + 1).sum())}
 
 
+def indexer_roofline(info, sel_ms, peaks):
+    """The selection stage (fold + indexer/top-k) against the FP8 tensor
+    peak.  The work is one score sweep's algorithmic FLOP, 2·128·Σ(pos+1),
+    divided by the stage's event time; the index rows it writes are reported
+    beside it.  There is no measured FP8 peak, so it is the measured
+    sustained bf16 peak times the nominal FP8/BF16 ratio (4.5 / 2.25)."""
+    flops = 2.0 * 128 * info["pairs"]
+    peak = 2.0 * peaks["bf16_tflops_sustained"]
+    achieved = flops / (sel_ms / 1e3) / 1e12
+    out_bytes = 4 * info["sum_sel"]
+    return {"stage": "select (fold + indexer/top-k)", "bound": "tensor", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_kind": f"fp8 = 2 x bf16 {peaks['source']} sustained (nominal ratio)", "flops_per_call": flops,
+            "index_out_bytes": out_bytes, "index_out_gbs": out_bytes / (sel_ms / 1e3) / 1e9}
+
+
 def attn_flops(wl, info):
     return 2.0 * wl.heads * (wl.dk + wl.dv) * info["sum_sel"]
 
@@ -568,6 +584,8 @@ def native(args):
         "gpu_launches": step_launches(wl) * args.steps,
         "clocks": clocks,
     }
+    if wl.idx_dtype == "e4m3":
+        res["stage_rooflines"] = {"indexer_topk": indexer_roofline(info, max_over_ranks(sel_ms, ws_n, dev), peaks)}
     tr = captured_traffic(wl.name, "attn_tc_kernel")
     if tr:
         res["roofline"]["traffic"] = tr["bytes_per_launch"]
