@@ -98,14 +98,26 @@ bool needs_scores(const dsa_seqs* s, const dsa_indexer_args* ia) {
     return !use_tc_indexer(s, ia) || use_split_select(s, ia);
 }
 
-// CTAs per row block for a score sweep: about two per SM in all, each over
-// at least four 256-key tiles.
-int score_tile_splits(const dsa_seqs* s) {
+int sm_count() {
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) {
         int v = 0;
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
     }
+    return sms;
+}
+
+// the fused selection (sampled score window, bitmask per row) runs
+bool use_fused_select(const dsa_seqs* s, const dsa_indexer_args* ia) {
+    return use_tc_indexer(s, ia) && !use_split_select(s, ia);
+}
+int64_t sel_words(const dsa_seqs* s) { return 8 * ((s->max_seqlen_k + 255) / 256); }
+int sel_ctas(const dsa_seqs* s) { return indexer_sel_ctas(indexer_blocks(s), sm_count()); }
+
+// CTAs per row block for a score sweep: about two per SM in all, each over
+// at least four 256-key tiles.
+int score_tile_splits(const dsa_seqs* s) {
+    const int sms = sm_count();
     const int64_t blocks = indexer_blocks(s) > 0 ? indexer_blocks(s) : 1;
     const int64_t max_tiles = (s->max_seqlen_k + 255) / 256;
     int64_t n = (2 * sms + blocks - 1) / blocks;
@@ -116,7 +128,7 @@ int score_tile_splits(const dsa_seqs* s) {
 }
 
 struct WsLayout {
-    size_t u, s_row, idx, scores, total;
+    size_t u, s_row, idx, scores, sel, total;
 };
 
 WsLayout ws_layout(const dsa_seqs* s, const dsa_indexer_args* ia, int32_t k, bool with_idx, bool with_scores) {
@@ -131,6 +143,10 @@ WsLayout ws_layout(const dsa_seqs* s, const dsa_indexer_args* ia, int32_t k, boo
     if (with_idx) off = align256(off + (size_t)s->total_q * (size_t)k * 4);
     L.scores = off;
     if (with_scores) off = align256(off + (size_t)s->total_q * (size_t)s->max_seqlen_k * 4);
+    // the fused selection's bitmask scratch: 128 rows of sel_words per CTA
+    L.sel = off;
+    if (with_idx && ia && use_fused_select(s, ia))
+        off = align256(off + (size_t)sel_ctas(s) * 128 * (size_t)sel_words(s) * 4);
     L.total = off;
     return L;
 }
@@ -279,6 +295,38 @@ int run_indexer_tc(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u,
     if (!make_map_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, ia->k_idx, 128, (uint64_t)s->total_k, 128, 128, 256))
         return DSA_ERR_CUDA;
     if (!launch_indexer_tc(a, st)) return DSA_ERR_CUDA;
+    return cuda_status();
+}
+
+// The fused selection: persistent CTAs, each with its slice of the bitmask
+// scratch at w + L.sel.
+int run_indexer_sel(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u, const float* s_row, int32_t k,
+                    int32_t* idx, int64_t ld_idx, uint32_t* sel_bits, StatusHdr* h, cudaStream_t st) {
+    IndexerTcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.sv = seq_view(s);
+    a.mode = 0;
+    a.total_q = s->total_q;
+    a.max_seqlen_q = s->max_seqlen_q;
+    a.s_row = s_row;
+    a.k_scale = ia->k_idx_scale;
+    a.k = k;
+    a.k_rows = ia->k_per_row;
+    a.idx = idx;
+    a.ld_idx = ld_idx;
+    a.tile_splits = 1;
+    a.st = h;
+    a.sel_bits = sel_bits;
+    a.sel_words = sel_words(s);
+    if (!make_map_2d(&a.tm_u, CU_TENSOR_MAP_DATA_TYPE_UINT8, u, 128, (uint64_t)s->total_q, 128, 128, 128))
+        return DSA_ERR_CUDA;
+    if (!make_map_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, ia->k_idx, 128, (uint64_t)s->total_k, 128, 128, 256))
+        return DSA_ERR_CUDA;
+    // every 16th key row: rows of 128 codes, 16 * 128 bytes apart
+    if (!make_map_2d(&a.tm_ks, CU_TENSOR_MAP_DATA_TYPE_UINT8, ia->k_idx, 128, (uint64_t)((s->total_k + 15) / 16),
+                     16 * 128, 128, 256))
+        return DSA_ERR_CUDA;
+    if (!launch_indexer_sel(a, sel_ctas(s), st)) return DSA_ERR_CUDA;
     return cuda_status();
 }
 
@@ -620,8 +668,8 @@ int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int
         return r;
     }
     if (use_tc_indexer(seqs, ia))
-        return run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, k, idx, ldi, nullptr, 0, 0, 0, hdr(ws),
-                              st);
+        return run_indexer_sel(seqs, ia, w + L.u, (const float*)(w + L.s_row), k, idx, ldi, (uint32_t*)(w + L.sel),
+                               hdr(ws), st);
     r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st, false);
     if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row);
     return r;

@@ -95,9 +95,18 @@ struct IndexerTcArgs {
     StatusHdr* st;
     CUtensorMap tm_u;       // folded query codes [total_q,128], box 128x128
     CUtensorMap tm_k;       // key codes [total_k,128], box 128x256
+    // the sampled-threshold selection (launch_indexer_sel) only:
+    uint32_t* sel_bits;     // per-CTA bitmask scratch, [ctas][128 rows][sel_words]
+    int64_t sel_words;      // 8 * ceil(max_seqlen_k / 256)
+    CUtensorMap tm_ks;      // every 16th key row [ceil(total_k/16),128], box 128x256
 };
 bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s);
 extern const int kIndexerRowsPerBlock;
+
+// The fused indexer / exact top-k with a sampled score window (prefill
+// shapes): a persistent grid of `ctas` CTAs, each with its own bitmask scratch.
+int indexer_sel_ctas(int64_t blocks, int sms);
+bool launch_indexer_sel(const IndexerTcArgs& a, int ctas, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // tcgen05 BF16 sparse MQA attention, 128 heads, dk 576, dv 512, CTA pairs.
