@@ -112,7 +112,9 @@ def test_selection_path_workspace(lib):
     """The selection path follows from the shapes alone, and so does the
     workspace.  Fewer 128-row blocks than SMs over > 2048 keys select in two launches
     through a score buffer of total_q x max_seqlen_k floats.  Otherwise the
-    prefill-shaped problem runs fused, with no score buffer."""
+    prefill-shaped problem runs fused, with no score buffer: each of its
+    persistent CTAs (at most one per SM; 148 without a GPU to ask) holds a
+    bitmask of 128 rows x 8 * ceil(max_seqlen_k / 256) words."""
     n = ctypes.c_size_t(0)
     ia = lib.dsa_indexer_args(lib.DSA_E4M3, 0x100000, 0x110000, lib.DSA_BF16, 0x200000, 0x300000, 0x310000)
 
@@ -130,7 +132,10 @@ def test_selection_path_workspace(lib):
     for b, tq, tk, mq, mk in split:
         assert size(b, tq, tk, mq, mk) >= tq * mk * 4 + tq * k * 4, (b, tq, tk)
     for b, tq, tk, mq, mk in fused:
-        assert size(b, tq, tk, mq, mk) < tq * k * 4 + tq * 256 + (1 << 20), (b, tq, tk)
+        ctas = min(148, b * ((mq + 127) // 128))
+        bits = ctas * 128 * 8 * ((mk + 255) // 256) * 4
+        got = size(b, tq, tk, mq, mk)
+        assert bits <= got < tq * k * 4 + tq * 256 + (1 << 20) + bits, (b, tq, tk)
 
 
 def test_backward_validation(lib):
