@@ -300,6 +300,8 @@ int run_indexer_tc(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u,
 
 // The fused selection: persistent CTAs, each with its slice of the bitmask
 // scratch at w + L.sel.
+constexpr size_t kWorkCounterOffset = 64;  // inside the 256-byte status header
+
 int run_indexer_sel(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u, const float* s_row, int32_t k,
                     int32_t* idx, int64_t ld_idx, uint32_t* sel_bits, StatusHdr* h, cudaStream_t st) {
     IndexerTcArgs a;
@@ -326,6 +328,9 @@ int run_indexer_sel(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u
     if (!make_map_2d(&a.tm_ks, CU_TENSOR_MAP_DATA_TYPE_UINT8, ia->k_idx, 128, (uint64_t)((s->total_k + 15) / 16),
                      16 * 128, 128, 256))
         return DSA_ERR_CUDA;
+    // the persistent CTAs take row blocks from a counter in the status header
+    a.work_counter = (uint32_t*)((uint8_t*)h + kWorkCounterOffset);
+    if (cudaMemsetAsync(a.work_counter, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
     if (!launch_indexer_sel(a, sel_ctas(s), st)) return DSA_ERR_CUDA;
     return cuda_status();
 }

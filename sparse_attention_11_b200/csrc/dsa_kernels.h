@@ -99,6 +99,7 @@ struct IndexerTcArgs {
     uint32_t* sel_bits;     // per-CTA bitmask scratch, [ctas][128 rows][sel_words]
     int64_t sel_words;      // 8 * ceil(max_seqlen_k / 256)
     CUtensorMap tm_ks;      // every 16th key row [ceil(total_k/16),128], box 128x256
+    uint32_t* work_counter; // row blocks handed out so far (zero at launch)
 };
 bool launch_indexer_tc(const IndexerTcArgs& a, cudaStream_t s);
 extern const int kIndexerRowsPerBlock;
