@@ -153,32 +153,30 @@ DSA_DEV void raw_scores(uint32_t* v, const float* scs, uint64_t srow2) {
 // Keys order like the scores.
 DSA_DEV uint32_t score_key(uint32_t raw) { return (uint32_t)__vimin_s32_relu((int)raw, (int)kInfKey); }
 
-// Add 1 to the shared-memory counter at `addr` when `bin` is not 0 (a
-// predicated reduction, so the 32 updates of a chunk need no branches).
-DSA_DEV void red_if(uint32_t addr, int bin) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.s32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(addr), "r"(bin)
-        : "memory");
-}
+// Add 1 to the shared-memory counter at `addr`.  Every key of a chunk is
+// counted (no predicate, no branch); keys that no decision needs (below the
+// window, past the causal limit, outside the bucket) go to bin 0, which no
+// decision reads.
+DSA_DEV void red_add(uint32_t addr) { asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory"); }
 
 // Histogram of 32 raw scores, bin = clamp((bits >> sh) + nc0, 0, 255) on the
 // raw bits (nc0 = -c0).  With c0 >= 0 every non-positive raw score lands in
 // bin 0 with the score +0, and with (kInfKey >> sh) - c0 >= 255 NaN lands in
-// bin 255 with +inf, so the bins are those of the score keys.  Bin 0 is not
-// counted (no decision needs it).  Columns past `lim` are skipped.  hbase is
-// the shared address of the row's bin 0; bin b is b * 512 bytes further.
+// bin 255 with +inf, so the bins are those of the score keys.  Columns past
+// `lim` go to bin 0.  hbase is the shared address of the row's bin 0; bin b is
+// b * 512 bytes further.
 DSA_DEV void hist_chunk(const uint32_t* v, int sh, int nc0, int lim, uint32_t hbase) {
     if (lim >= 31) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int bin = __viaddmin_s32_relu((int)v[i] >> sh, nc0, 255);
-            red_if(hbase + (bin << 9), bin);
+            red_add(hbase + (bin << 9));
         }
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int bin = __viaddmin_s32_relu((int)v[i] >> sh, nc0, 255);
-            red_if(hbase + (bin << 9), i <= lim ? bin : 0);
+            red_add(hbase + ((i <= lim ? bin : 0) << 9));
         }
     }
 }
@@ -186,23 +184,26 @@ DSA_DEV void hist_chunk(const uint32_t* v, int sh, int nc0, int lim, uint32_t hb
 // The same with the zero score in a bin of its own: bin 0 holds exactly the
 // score 0 (every non-positive raw score), bin 1 the positive scores below the
 // window, bins 2..254 the window, bin 255 the rest.  For blocks with rows
-// whose K-th score may be 0 or close to it.
+// whose K-th score may be 0 or close to it.  Bin 0 is not read either (a K-th
+// score of 0 is a single-valued bucket, taken in index order), so the columns
+// past `lim` go there too.
 DSA_DEV void hist_chunk_z(const uint32_t* v, int sh, int nc0, int lim, uint32_t hbase) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int t = ((int)v[i] >> sh) + nc0;
         const int bin = __vimin_s32_relu(max(t, min((int)v[i], 1)), 255);
-        red_if(hbase + (bin << 9), i <= lim ? bin : 0);
+        red_add(hbase + ((i <= lim ? bin : 0) << 9));
     }
 }
 
-// Histogram of the keys inside a bucket [lo, lo + w): bin 1 + ((key - lo) >> sh).
+// Histogram of the keys inside a bucket [lo, lo + w): bin 1 + ((key - lo) >> sh);
+// the other keys go to bin 0.
 DSA_DEV void ref_chunk(const uint32_t* v, uint32_t lo, uint32_t w, int sh, int lim, uint32_t hbase) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const uint32_t d = score_key(v[i]) - lo;
-        const int bin = 1 + (int)(d >> sh);
-        red_if(hbase + (bin << 9), (d < w && i <= lim) ? bin : 0);
+        const int bin = (d < w && i <= lim) ? 1 + (int)(d >> sh) : 0;
+        red_add(hbase + (bin << 9));
     }
 }
 
