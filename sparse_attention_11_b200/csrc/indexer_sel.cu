@@ -112,6 +112,7 @@ struct RowState {
     int pad[2];
 };
 static_assert(sizeof(RowState) == 64, "RowState layout");
+static_assert(sizeof(Bars) <= 256, "barrier block");
 
 // ---------------------------------------------------------------------------
 // packed fp32 pairs (sm_100a f32x2 arithmetic; each lane rounds like the
@@ -332,7 +333,7 @@ DSA_DEV uint32_t staged(const uint32_t* row, int i, uint32_t lane) {
 // After the emission sweep: a listed bucket (at most kListCap keys with their
 // score keys, in shared memory) keeps its `need` best (score key desc, index
 // asc); the others are cleared from the row's bitmask.  One warp per row.
-__device__ __noinline__ void resolve_lists(const IndexerTcArgs& a, uint32_t* scratch, const RowState* rstate,
+__device__ __noinline__ void resolve_lists(const int64_t sel_words, uint32_t* scratch, const RowState* rstate,
                                            const uint2* list, const uint32_t* lcnt, int ew, uint32_t lane, int nrows) {
     constexpr int kRowsPerWarp = BM / EPI_WARPS;
     for (int j = 0; j < kRowsPerWarp; ++j) {
@@ -343,7 +344,7 @@ __device__ __noinline__ void resolve_lists(const IndexerTcArgs& a, uint32_t* scr
         const uint32_t need = rr.need;
         // entries name keys of this row (0..pos): checked before the bitmask is touched
         const uint32_t nk = (uint32_t)rr.pos + 1;
-        uint32_t* srow_bits = scratch + (size_t)rr_i * a.sel_words;
+        uint32_t* srow_bits = scratch + (size_t)rr_i * sel_words;
         const uint32_t C = min(lcnt[rr_i], (uint32_t)kListCap);
         const uint2 e0 = lane < C ? list[lane * BM + rr_i] : make_uint2(0u, 0u);
         const uint2 e1 = lane + 32 < C ? list[(lane + 32) * BM + rr_i] : make_uint2(0u, 0u);
@@ -434,22 +435,23 @@ __device__ __noinline__ void decide_s2(RowState& rw, const uint32_t* hrow) {
 // The finish: one warp per row turns the row's bitmask into its ascending
 // index row (lanes take eight consecutive words each, indices are staged in
 // shared memory and written out coalesced), -1 after the K_t-th.
-__device__ __noinline__ void finish_rows(const IndexerTcArgs& a, const uint32_t* scratch, const RowState* rstate,
-                                         int* stg, int64_t t_first, int nrows, int ew, uint32_t lane,
-                                         volatile int* abort) {
+__device__ __noinline__ void finish_rows(int32_t* idx, int64_t ld_idx, const int k_out, const int64_t sel_words,
+                                         StatusHdr* st, const uint32_t* scratch, const RowState* rstate, int* stg,
+                                         int64_t t_first, int nrows, int ew, uint32_t lane, volatile int* abort) {
     constexpr int kRowsPerWarp = BM / EPI_WARPS;
+    const int kcap = min(kStageInts, k_out);  // indices past it go straight to memory
     for (int j = 0; j < kRowsPerWarp; ++j) {
         const int rr_i = ew * kRowsPerWarp + j;
         if (rr_i >= nrows || __any_sync(0xffffffffu, *abort != 0)) break;
         const int kind = rstate[rr_i].kind, pos = rstate[rr_i].pos, kt = rstate[rr_i].kt;
         const int64_t tr = t_first + rr_i;
-        int32_t* out = a.idx + tr * a.ld_idx;
+        int32_t* out = idx + tr * ld_idx;
         if (kind != ROW_SEL) {
             const int n = kind == ROW_PREFIX ? pos + 1 : 0;
-            for (int jj = lane; jj < a.k; jj += 32) out[jj] = jj < n ? jj : -1;
+            for (int jj = lane; jj < k_out; jj += 32) out[jj] = jj < n ? jj : -1;
             continue;
         }
-        const uint32_t* srow_bits = scratch + (size_t)rr_i * a.sel_words;
+        const uint32_t* srow_bits = scratch + (size_t)rr_i * sel_words;
         const int nw = (pos >> 5) + 1;
         int written = 0;
         for (int gb = 0; gb < nw; gb += 256) {
@@ -481,15 +483,15 @@ __device__ __noinline__ void finish_rows(const IndexerTcArgs& a, const uint32_t*
                 while (sbits) {
                     const int i = __ffs(sbits) - 1;
                     sbits &= sbits - 1;
-                    if (off < kStageInts) stg[off] = kb + i;
-                    else if (off < a.k) out[off] = kb + i;
+                    if (off < kcap) stg[off] = kb + i;
+                    else if (off < k_out) out[off] = kb + i;
                     ++off;
                 }
             }
             written += total;
         }
         __syncwarp();
-        const int nstg = min(written, min(kStageInts, a.k));
+        const int nstg = min(written, kcap);
         if ((((uintptr_t)out) & 15) == 0) {
             const int n4 = nstg >> 2;
             for (int jj = lane; jj < n4; jj += 32) ((int4*)out)[jj] = ((const int4*)stg)[jj];
@@ -497,8 +499,8 @@ __device__ __noinline__ void finish_rows(const IndexerTcArgs& a, const uint32_t*
         } else {
             for (int jj = lane; jj < nstg; jj += 32) out[jj] = stg[jj];
         }
-        for (int jj = written + (int)lane; jj < a.k; jj += 32) out[jj] = -1;
-        if (written != kt && !*abort && lane == 0) report(a.st, DSA_ERR_INDEX, -3000000 - tr);
+        for (int jj = written + (int)lane; jj < k_out; jj += 32) out[jj] = -1;
+        if (written != kt && !*abort && lane == 0) report(st, DSA_ERR_INDEX, -3000000 - tr);
         __syncwarp();
     }
 }
@@ -834,7 +836,7 @@ __global__ void __maxnreg__(96) indexer_sel_kernel(const __grid_constant__ Index
                     }
                     // ---- listed buckets keep their `need` best ----
                     asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");  // every list entry is in
-                    resolve_lists(a, scratch, rstate, (const uint2*)(smem + OFF_LIST), lcnt, ew, lane, nrows);
+                    resolve_lists(a.sel_words, scratch, rstate, (const uint2*)(smem + OFF_LIST), lcnt, ew, lane, nrows);
                     __threadfence_block();
                     next = SK_STOP;
                 } else {
@@ -919,7 +921,8 @@ __global__ void __maxnreg__(96) indexer_sel_kernel(const __grid_constant__ Index
             __threadfence_block();
             asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory");  // every bitmask word is final
             // ---- finish: bitmask -> ascending indices, staged in the region ----
-            finish_rows(a, scratch, rstate, (int*)(smem + OFF_R) + ew * kStageInts, t_first, nrows, ew, lane, abort);
+            finish_rows(a.idx, a.ld_idx, a.k, a.sel_words, st, scratch, rstate, (int*)(smem + OFF_R) + ew * kStageInts,
+                        t_first, nrows, ew, lane, abort);
         }
     }
     // drain on abort: loads and MMAs in flight must land before TMEM and the CTA go away

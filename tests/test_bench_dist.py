@@ -61,15 +61,15 @@ def test_reference_arm_prints_only_on_rank0():
 
 def test_indexer_roofline_arithmetic():
     """The selection stage's roofline: one sweep's 2·128·Σ(pos+1) FLOP per
-    event time, against twice the measured sustained bf16 peak."""
+    event time, against the FP8 GEMM peak measured in the same run."""
     sys.path.insert(0, ROOT)
     import bench
     from sparse_attention_11_b200 import workloads as W
     wl = W.custom("probe", (1000,), (1000,), base="prefill_l8192", k=100)
     info = bench.workload_info(wl)
     assert info["pairs"] == 1000 * 1001 // 2 and info["sum_sel"] == 100 * 101 // 2 + 900 * 100
-    peaks = {"hbm_gbs": 1.0, "bf16_tflops": 10.0, "bf16_tflops_sustained": 5.0, "source": "test"}
-    r = bench.indexer_roofline(info, 2.0, peaks)
+    fp8 = {"fp8_tflops": 10.0, "how": "test"}
+    r = bench.indexer_roofline(info, 2.0, fp8)
     assert r["peak"] == 10.0
     assert abs(r["achieved"] - 2 * 128 * 500500 / 2e-3 / 1e12) < 1e-12
     assert abs(r["frac"] - r["achieved"] / 10.0) < 1e-15

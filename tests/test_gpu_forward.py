@@ -49,6 +49,13 @@ def _consistency(prob, rows_begin, rows_count):
     assert np.array_equal(a, b), f"fused selection differs from topk(scores) in {np.any(a != b, axis=1).sum()} rows"
 
 
+def _boundary_rows(wl):
+    """Rows at the positions where the selection changes character: pos = k-1
+    (the last row that keeps its whole prefix), k, k+1."""
+    T, k = wl.total_q, wl.k
+    return np.array([p for p in (k - 1, k, k + 1) if 0 <= p < T], dtype=np.int64)
+
+
 def _run(name, n_sel_rows, n_attn_rows, consistency_ranges):
     wl = W.WORKLOADS[name] if isinstance(name, str) else name
     inp, prob = make(wl)
@@ -68,7 +75,8 @@ def _run(name, n_sel_rows, n_attn_rows, consistency_ranges):
         K = min(wl.k, int(pos[r]) + 1)
         assert np.all(g_idx[r, K:] == -1) and np.all(np.diff(g_idx[r, :K]) > 0)
         assert g_idx[r, :K].min() >= 0 and g_idx[r, :K].max() <= pos[r]
-    arows = stratified_rows(T, n_attn_rows, seed=2)
+    arows = np.unique(np.concatenate([stratified_rows(T, n_attn_rows, seed=2), _boundary_rows(wl)])) \
+        if wl.batch == 1 else stratified_rows(T, n_attn_rows, seed=2)
     g_idx_a = g_idx_all[torch.from_numpy(arows).cuda()].cpu().numpy()
     o, olse = oracle_attention_rows(inp, arows, g_idx_a)
     g, glse = gpu_out_rows(prob, arows)
@@ -115,11 +123,35 @@ def test_forward_decode_b64():
 
 
 def test_forward_prefill_l32768():
-    _run("prefill_l32768", 256, 32, [(0, 128), (16384, 256), (32768 - 128, 128)])
+    _run("prefill_l32768", 256, 128, [(0, 128), (16384, 256), (32768 - 128, 128)])
 
 
 def test_forward_prefill_l131072():
-    _run("prefill_l131072", 256, 24, [(131072 - 128, 128), (65536, 128)])
+    _run("prefill_l131072", 256, 128, [(131072 - 128, 128), (65536, 128)])
+
+
+def test_fused_selection_matches_oracle_topk_l32768():
+    """The fused selection at L=32768 against the oracle's top-k of the GPU's
+    own scores (dsa_index_scores), row by row: identical index sets on 256
+    rows spread over every position band plus the rows at pos = k-1, k, k+1
+    (the comparison does not go through dsa_topk)."""
+    wl = W.WORKLOADS["prefill_l32768"]
+    inp, prob = make(wl)
+    dsa.dsa_select(prob.seqs, prob.ia, wl.k, prob.idx, prob.ws)
+    prob.check("select")
+    rows = np.unique(np.concatenate([stratified_rows(wl.total_q, 256, seed=3), _boundary_rows(wl)]))
+    ld = prob.seqs.max_seqlen_k
+    sc = torch.empty((1, ld), dtype=torch.float32, device="cuda")
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_INDEX_SCORES, prob.seqs, 0, prob.ia))
+    g_sc = np.empty((len(rows), ld), dtype=np.float32)
+    for i, r in enumerate(rows):
+        dsa.dsa_index_scores(prob.seqs, prob.ia, int(r), 1, sc, ws)
+        g_sc[i] = sc[0].cpu().numpy()
+    dsa.check_device_status(ws, "index_scores")
+    _, pos = inp.key_base_pos(rows)
+    o_idx = oracle.topk(g_sc, pos + 1, wl.k)
+    g_idx = prob.idx[torch.from_numpy(rows).cuda()].cpu().numpy()
+    sets_equal(g_idx, o_idx, pos + 1, wl.k)
 
 
 @pytest.mark.parametrize("name", ["prefill_l8192", "batched"])
