@@ -64,6 +64,11 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
     ap.add_argument("--probe-fp8-peak", action="store_true",
                     help="only measure the dense FP8 (e4m3) GEMM peak of this GPU (burst and sustained) and print it")
+    ap.add_argument("--profile-case", choices=["select", "decode-small"],
+                    help="run a lean case for a profiler (no timing line): 'select' = dsa_select on --workload with "
+                         "the indexer inputs only; 'decode-small' = decode select + attention, 64 sequences with "
+                         "contexts 16K-24K")
+    ap.add_argument("--reps", type=int, default=3, help="calls of the --profile-case")
     return ap.parse_args()
 
 
@@ -737,8 +742,51 @@ def reference(args):
     print(json.dumps(res), flush=True)
 
 
+def profile_case(args):
+    """Lean cases for profiler captures: the device holds only what the
+    captured kernels read and write (a few GB at most)."""
+    import torch
+    from sparse_attention_11_b200 import dsa, workloads as W
+    from sparse_attention_11_b200.problem import DeviceProblem
+    if args.profile_case == "select":
+        wl = W.WORKLOADS[args.workload]
+        s = wl.seed
+        cu_q = np.concatenate([[0], np.cumsum(wl.seqlens_q)]).astype(np.int64)
+        cu_k = np.concatenate([[0], np.cumsum(wl.seqlens_k)]).astype(np.int64)
+        qf = W.bf16_bits_to_f32(W.to_bf16_bits(W._sub_rng(s, "q_idx").standard_normal((wl.total_q, 128),
+                                                                                        dtype=np.float32)))
+        kf = W.bf16_bits_to_f32(W.to_bf16_bits(W._indexer_keys(W._sub_rng(s, "k_idx"), wl.total_k)))
+        q_idx, q_sc = W.quantize_e4m3_rows(qf)
+        k_idx, k_sc = W.quantize_e4m3_rows(kf)
+        Wf = W._sub_rng(s, "W_index").standard_normal((128, 128), dtype=np.float32) / np.float32(math.sqrt(128.0))
+        Wb = torch.from_numpy(W.to_bf16_bits(Wf).view(np.int16)).view(torch.bfloat16).cuda()
+        seqs = dsa.Seqs(cu_q, cu_k, device=torch.device("cuda"))
+        ia = dsa.indexer_args(torch.from_numpy(q_idx).cuda(), torch.from_numpy(q_sc).cuda(), Wb,
+                              torch.from_numpy(k_idx).cuda(), torch.from_numpy(k_sc).cuda())
+        ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, seqs, wl.k, ia))
+        idx = torch.empty((wl.total_q, wl.k), dtype=torch.int32, device="cuda")
+        for _ in range(args.reps):
+            dsa.dsa_select(seqs, ia, wl.k, idx, ws)
+        torch.cuda.synchronize()
+        dsa.check_device_status(ws, "profile case select")
+    else:
+        rng = np.random.default_rng(0)
+        ctx = tuple(int(x) for x in rng.integers(16384, 24577, size=64))
+        wl = W.custom("decode_b64_ctx16k_24k", (1,) * 64, ctx, base="decode_b64")
+        prob = DeviceProblem(W.generate(wl, device="cuda"))
+        for _ in range(args.reps):
+            dsa.dsa_select(prob.seqs, prob.ia, wl.k, prob.idx, prob.ws)
+            dsa.dsa_sparse_attn(prob.seqs, prob.aa, prob.idx, wl.k, prob.ws)
+        torch.cuda.synchronize()
+        prob.check("profile case decode-small")
+    print("profile case done:", args.profile_case, wl.name, flush=True)
+
+
 def main():
     args = parse()
+    if args.profile_case:
+        profile_case(args)
+        return
     if args.probe_fp8_peak:
         print(json.dumps(fp8_peak(burst_reps=10, sustained_s=4.0)), flush=True)
         return
