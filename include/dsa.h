@@ -154,7 +154,8 @@ DSA_API int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const ds
  * F32:  u_out float [total_q,128] = fp32(q W); s_row_out[t] = 1.
  * E4M3: u' = q8 W (q8 the decoded codes), s_u = fp32(amax|u'|/448) (1 when
  *       amax = 0), u_out = e4m3 codes of fp32(u'/s_u) (round to nearest even,
- *       saturating), s_row_out[t] = fp32(q_idx_scale[t] * s_u).           */
+ *       saturating), s_row_out[t] = fp32(q_idx_scale[t] * s_u).
+ * u_out must be 16-byte aligned (DSA_ERR_INVALID_ARG otherwise).          */
 DSA_API int dsa_fold(const dsa_seqs* seqs, const dsa_indexer_args* ia, void* u_out, float* s_row_out,
              void* ws, size_t ws_bytes, dsa_stream_t stream);
 
@@ -262,9 +263,14 @@ DSA_API int dsa_indexer_kl(const dsa_seqs* seqs, const float* q_idx, int64_t q_s
  *   (total_q x max_seqlen_k floats) fits in 8 GiB, the selection runs in two
  *   launches instead.  This is the case of a query chunk over a long prefix.
  *   The first launch is a score sweep that splits each block's key range over
- *   several CTAs; the second is the radix top-k of dsa_topk.  The scores pass
- *   through the workspace, and the result is the same.
- * - Decode-shaped or F32 problems use the scan + radix top-k. */
+ *   several CTAs; the second selects per row from the scores (as below for
+ *   decode).  The scores pass through the workspace, and the result is the
+ *   same.
+ * - Decode-shaped (max_seqlen_q < 64) or F32 problems scan the keys with
+ *   CUDA cores into a workspace score buffer, then select per row: a
+ *   histogram of the row's scores in 4096 bins of 1/16 binade, the bin of
+ *   the k-th score refined on chip, one placement pass.
+ * All paths give the same indices. */
 DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
                        int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
@@ -276,7 +282,9 @@ DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t
  * it is a deployment convenience of this library.
  *
  * Same result as dsa_select.  Only prefill-shaped E4M3 inputs
- * (max_seqlen_q >= 64, the fused tensor-core indexer) are served, with at
+ * (max_seqlen_q >= 64) are served, always by the fused tensor-core indexer
+ * with the scratch-free radix selection (no bitmask scratch; slower than
+ * dsa_select's selection at long sequences, the same indices), with at
  * most 32768 query rows in total; more rows return DSA_ERR_WORKSPACE, other
  * shapes DSA_ERR_UNSUPPORTED, and nothing is launched.
  *

@@ -336,7 +336,8 @@ int run_indexer_sel(const dsa_seqs* s, const dsa_indexer_args* ia, const void* u
 }
 
 int run_topk(const dsa_seqs* s, const float* scores, int64_t ld, int64_t row_begin, int64_t row_count, int32_t k,
-             int32_t* idx, int64_t ld_idx, StatusHdr* h, cudaStream_t st, const int32_t* k_rows = nullptr) {
+             int32_t* idx, int64_t ld_idx, StatusHdr* h, cudaStream_t st, const int32_t* k_rows = nullptr,
+             bool nonneg = false) {
     TopkArgs a;
     a.k_rows = k_rows;
     a.sv = seq_view(s);
@@ -348,7 +349,8 @@ int run_topk(const dsa_seqs* s, const float* scores, int64_t ld, int64_t row_beg
     a.idx = idx;
     a.ld_idx = ld_idx;
     a.st = h;
-    launch_topk_rows(a, st);
+    if (nonneg) launch_topk_hist(a, st);  // the selection's own ReLU scores
+    else launch_topk_rows(a, st);
     return cuda_status();
 }
 
@@ -461,7 +463,7 @@ int dsa_fold(const dsa_seqs* seqs, const dsa_indexer_args* ia, void* u_out, floa
              dsa_stream_t stream) {
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
-    if (!r && seqs->total_q && (!u_out || !s_row_out)) r = DSA_ERR_INVALID_ARG;
+    if (!r && seqs->total_q && (!u_out || !s_row_out || !aligned(u_out, 16))) r = DSA_ERR_INVALID_ARG;
     if (!r) r = check_ws(ws, ws_bytes, kHdr);
     if (r) return r;
     return run_fold(seqs, ia, u_out, s_row_out, (cudaStream_t)stream);
@@ -669,14 +671,14 @@ int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int
         // scores past each row's position are left unwritten: the top-k reads 0..pos
         r = run_indexer_tc(seqs, ia, w + L.u, (const float*)(w + L.s_row), 1, 0, nullptr, 0, sc, ld, 0, seqs->total_q,
                            hdr(ws), st);
-        if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row);
+        if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row, true);
         return r;
     }
     if (use_tc_indexer(seqs, ia))
         return run_indexer_sel(seqs, ia, w + L.u, (const float*)(w + L.s_row), k, idx, ldi, (uint32_t*)(w + L.sel),
                                hdr(ws), st);
     r = run_scores_simt(seqs, ia, w + L.u, (const float*)(w + L.s_row), 0, seqs->total_q, sc, ld, hdr(ws), st, false);
-    if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row);
+    if (!r) r = run_topk(seqs, sc, ld, 0, seqs->total_q, k, idx, ldi, hdr(ws), st, ia->k_per_row, true);
     return r;
 }
 }  // namespace

@@ -47,6 +47,9 @@ struct TopkArgs {
     StatusHdr* st;
 };
 void launch_topk_rows(const TopkArgs& a, cudaStream_t s);
+// The same selection for non-negative scores (ReLU scores, +inf for NaN),
+// by a histogram of 1/16 binade bins, then the boundary bin's keys on chip.
+void launch_topk_hist(const TopkArgs& a, cudaStream_t s);
 
 struct AttnF32Args {
     int heads;

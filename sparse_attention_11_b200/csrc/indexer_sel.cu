@@ -9,32 +9,36 @@
 // scores (ties to the lower key index).  The L x L scores never leave the SM.
 //
 // Work unit: a block of 128 consecutive queries of one sequence.  The grid is
-// persistent (one CTA per SM); CTA i takes blocks i, 2G-1-i, 2G+i, ... of the
-// heaviest-first order.  10 warps:
+// persistent (one CTA per SM); CTAs take blocks in heaviest-first order from
+// an atomic counter in the workspace.  18 warps:
 //   warp 0      TMA producer: the block's folded queries (128 x 128 e4m3),
-//               key tiles of 256 x 128 e4m3 and their fp32 scales
+//               key tiles of 256 x 128 e4m3 and their fp32 scales (own ring)
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma kind::f8f6f4,
 //               M=128 N=256, fp32 accumulators in two TMEM buffers
-//   warps 2..9  epilogue: two threads per query row, one per 128-column half
-//               of each tile; the score is ReLU((dot * s_k) * s_row)
+//   warps 2..17 epilogue: four threads per query row (its TMEM lane), one per
+//               64-column quarter of each tile; the score is
+//               ReLU((dot * s_k) * s_row), formed on packed f32x2 pairs
 //
 // Sweeps of one block (the MMAs are recomputed in each):
 //   S1, S2  over a sample of the common causal prefix (every 16th key): a
 //           per-row histogram of the sample's scores, by binade (S1) and then
-//           at 1/64 binade around the binade holding the sample's rank
-//           K_t * n_sample / n_keys (S2).  This estimates each row's K-th score.
-//   H       over all causal keys: a per-row histogram at 1/128 binade over
-//           two binades around the estimate (rows whose estimate is zero
-//           histogram the zero score and the denormals exactly).  The bin
-//           holding the K-th score is the row's bucket [lo, hi).
+//           at 1/64 binade (S2).  The ranks r -/+ (4 sqrt(r) + 1) around the
+//           row's sample rank r = K_t * n_sample / n_keys bound its K-th score.
+//   H       over all causal keys: a per-row histogram of 256 bins spanning
+//           that band, 1/128 binade or coarser (rows whose band reaches zero
+//           keep the score 0 in a bin of its own).  The bin holding the K-th
+//           score is the row's bucket [lo, hi).
 //   REF     (rare) when a bucket is too large to resolve, a further histogram
 //           of the keys inside it at 256 finer bins.
 //   E       over all causal keys: a bitmask per row of the keys at or above
 //           lo (keys at or above hi are always kept), written to a per-CTA
 //           scratch.  A bucket of a single score value takes its first `need`
-//           keys in index order (the two threads of a row trade their per-tile
-//           counts); a bucket of several values (at most kListCap keys) is
-//           listed on chip with the scores, and its losers are cleared after.
+//           keys in index order (the four threads of a row trade their
+//           per-tile counts); a bucket of several values (at most kListCap
+//           keys) is listed on chip with the scores, and its losers are
+//           cleared after.
+// Histogram updates are unpredicated shared-memory reductions: keys that no
+// row counts go to bin 0, which no decision reads.
 // Finish: one warp per row turns the bitmask into the ascending index row.
 #include "dsa_kernels.h"
 

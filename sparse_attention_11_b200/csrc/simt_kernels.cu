@@ -15,20 +15,124 @@
 namespace dsa {
 
 // ---------------------------------------------------------------------------
-// a1: fold.  Thread j of a 128-thread CTA keeps column j of W in registers
-// and folds up to FOLD_ROWS query rows (fewer when there are few rows, so
-// that the CTAs cover the GPU): u_j = sum_i q_i W[i][j] (fp32 FMA chain).
+// a1: fold.  u_j = sum_i q_i W[i][j], an fp32 FMA chain in i = 0..127 for
+// every output.  A CTA of FOLD_WARPS warps loads W once (fp32, 64 KB of
+// shared memory) and folds groups of FOLD_WARPS * RPW rows: warp w takes RPW
+// consecutive rows, lane l the columns 4l..4l+3 of each, so every step i is
+// one 16-byte read of W[i][4l..4l+3], RPW/4 broadcast 16-byte reads of the
+// rows' q_i (stored transposed) and 4 * RPW FMAs.  With many rows the grid is
+// two CTAs per SM, each looping over row groups.
 // E4M3: s_u = amax/448 (IEEE division), codes = e4m3_rn_satfinite(u_j / s_u),
-// s_row = s_q * s_u.
+// s_row = s_q * s_u.  The row's amax is a warp reduction; its codes are one
+// 128-byte store.  Short query sets (decode) use fold_cols_kernel instead:
+// thread j keeps column j of W in registers, one CTA per few rows, so the
+// CTAs cover the GPU without each loading all of W into shared memory.
 // ---------------------------------------------------------------------------
-constexpr int FOLD_ROWS = 32;
+constexpr int FOLD_WARPS = 8;
+constexpr int FOLD_COL_ROWS = 32;  // fold_cols_kernel: rows per CTA at most
 
 __device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
     __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
     return __half2float(__half(h));
 }
 
-__global__ void __launch_bounds__(128) fold_kernel(int64_t T, int idx_dtype, const void* __restrict__ q_idx,
+template <int RPW>
+constexpr uint32_t fold_smem_bytes() {
+    return 128 * 128 * 4 + FOLD_WARPS * 128 * (RPW < 4 ? 4 : RPW) * 4;  // W, then per warp q^T [128][max(RPW,4)]
+}
+
+template <int RPW>
+__global__ void __launch_bounds__(FOLD_WARPS * 32) fold_kernel(FoldArgs a) {
+    constexpr int QW = RPW < 4 ? 4 : RPW;  // row slots of the transposed q (16-byte reads)
+    extern __shared__ __align__(16) float fold_sm[];
+    float* ws = fold_sm;                                            // [128][128]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* qt = fold_sm + 128 * 128 + warp * 128 * QW;              // this warp's [128][QW]
+    if (a.w_dtype == DSA_F32) {
+        for (int e = threadIdx.x; e < 128 * 32; e += FOLD_WARPS * 32)
+            ((float4*)ws)[e] = __ldg((const float4*)a.W + e);
+    } else {
+        for (int e = threadIdx.x; e < 128 * 16; e += FOLD_WARPS * 32) {
+            const uint4 v = __ldg((const uint4*)a.W + e);  // 8 bf16
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            float4 lo, hi;
+            lo.x = __uint_as_float(w4[0] << 16), lo.y = __uint_as_float(w4[0] & 0xFFFF0000u);
+            lo.z = __uint_as_float(w4[1] << 16), lo.w = __uint_as_float(w4[1] & 0xFFFF0000u);
+            hi.x = __uint_as_float(w4[2] << 16), hi.y = __uint_as_float(w4[2] & 0xFFFF0000u);
+            hi.z = __uint_as_float(w4[3] << 16), hi.w = __uint_as_float(w4[3] & 0xFFFF0000u);
+            ((float4*)ws)[2 * e] = lo;
+            ((float4*)ws)[2 * e + 1] = hi;
+        }
+    }
+    __syncthreads();
+    const int64_t groups = (a.T + FOLD_WARPS * RPW - 1) / (FOLD_WARPS * RPW);
+    for (int64_t gi = blockIdx.x; gi < groups; gi += gridDim.x) {
+        const int64_t r0 = (gi * FOLD_WARPS + warp) * RPW;
+        if (r0 >= a.T) continue;
+        __syncwarp();
+        // this warp's rows, transposed: qt[i][rr] = q[r0 + rr][i] (0 past T)
+#pragma unroll
+        for (int rr = 0; rr < QW; ++rr) {
+            const int64_t r = r0 + rr;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int i = c * 32 + lane;
+                float v = 0.f;
+                if (rr < RPW && r < a.T)
+                    v = a.idx_dtype == DSA_F32 ? __ldg((const float*)a.q_idx + r * 128 + i)
+                                               : e4m3_to_f32(((const uint8_t*)a.q_idx)[r * 128 + i]);
+                qt[i * QW + rr] = v;
+            }
+        }
+        __syncwarp();
+        float acc[RPW][4];
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[rr][c] = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < 128; ++i) {
+            const float4 w4 = *(const float4*)(ws + i * 128 + 4 * lane);
+            float qv[QW];
+#pragma unroll
+            for (int rr = 0; rr < QW; rr += 4) {
+                const float4 q4 = *(const float4*)(qt + i * QW + rr);
+                qv[rr] = q4.x, qv[rr + 1] = q4.y, qv[rr + 2] = q4.z, qv[rr + 3] = q4.w;
+            }
+#pragma unroll
+            for (int rr = 0; rr < RPW; ++rr) {
+                acc[rr][0] = fmaf(qv[rr], w4.x, acc[rr][0]);
+                acc[rr][1] = fmaf(qv[rr], w4.y, acc[rr][1]);
+                acc[rr][2] = fmaf(qv[rr], w4.z, acc[rr][2]);
+                acc[rr][3] = fmaf(qv[rr], w4.w, acc[rr][3]);
+            }
+        }
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr) {
+            const int64_t r = r0 + rr;
+            if (r >= a.T) break;
+            if (a.idx_dtype == DSA_F32) {
+                ((float4*)a.u_out)[r * 32 + lane] = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+                if (lane == 0) a.s_row_out[r] = 1.0f;
+                continue;
+            }
+            float m = fmaxf(fmaxf(fabsf(acc[rr][0]), fabsf(acc[rr][1])), fmaxf(fabsf(acc[rr][2]), fabsf(acc[rr][3])));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const float s_u = m == 0.f ? 1.0f : __fdiv_rn(m, 448.0f);
+            uint32_t codes = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float y = m == 0.f ? 0.f : __fdiv_rn(acc[rr][c], s_u);
+                codes |= (uint32_t)(uint8_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3) << (8 * c);
+            }
+            ((uint32_t*)a.u_out)[r * 32 + lane] = codes;
+            if (lane == 0) a.s_row_out[r] = __fmul_rn(__ldg(a.q_scale + r), s_u);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128) fold_cols_kernel(int64_t T, int idx_dtype, const void* __restrict__ q_idx,
                                                    const float* __restrict__ q_scale, int w_dtype,
                                                    const void* __restrict__ W, void* __restrict__ u_out,
                                                    float* __restrict__ s_row_out, int rows_per_cta) {
@@ -74,14 +178,33 @@ __global__ void __launch_bounds__(128) fold_kernel(int64_t T, int idx_dtype, con
     }
 }
 
+template <int RPW>
+static void launch_fold_t(const FoldArgs& a, int64_t max_ctas, cudaStream_t s) {
+    constexpr uint32_t smem = fold_smem_bytes<RPW>();
+    cudaFuncSetAttribute(fold_kernel<RPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int64_t grid = (a.T + FOLD_WARPS * RPW - 1) / (FOLD_WARPS * RPW);
+    if (grid > max_ctas) grid = max_ctas;
+    fold_kernel<RPW><<<(unsigned)grid, FOLD_WARPS * 32, smem, s>>>(a);
+}
+
 void launch_fold(const FoldArgs& a, cudaStream_t s) {
     if (a.T <= 0) return;
-    // about four CTAs per SM of a B200 before a CTA takes more than one row
+    // many rows: 8 (or 2) per warp, at most two persistent CTAs per SM of a
+    // B200 (W is loaded once per CTA)
+    if (a.T >= 148 * FOLD_WARPS * 8) {
+        launch_fold_t<8>(a, 2 * 148, s);
+        return;
+    }
+    if (a.T >= 1024) {
+        launch_fold_t<2>(a, 2 * 148, s);
+        return;
+    }
+    // few rows (decode): about four CTAs per SM before a CTA takes more than one row
     int64_t rows = (a.T + 148 * 4 - 1) / (148 * 4);
-    if (rows > FOLD_ROWS) rows = FOLD_ROWS;
+    if (rows > FOLD_COL_ROWS) rows = FOLD_COL_ROWS;
     const int64_t grid = (a.T + rows - 1) / rows;
-    fold_kernel<<<(unsigned)grid, 128, 0, s>>>(a.T, a.idx_dtype, a.q_idx, a.q_scale, a.w_dtype, a.W, a.u_out, a.s_row_out,
-                                               (int)rows);
+    fold_cols_kernel<<<(unsigned)grid, 128, 0, s>>>(a.T, a.idx_dtype, a.q_idx, a.q_scale, a.w_dtype, a.W, a.u_out,
+                                                    a.s_row_out, (int)rows);
 }
 
 // ---------------------------------------------------------------------------
@@ -244,6 +367,64 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+constexpr int TOPK_BATCH = 8;  // 32-key rows of a warp's range loaded before any is used
+
+// Index range of each warp in the emission: contiguous, a multiple of 32.
+__device__ __forceinline__ int64_t topk_span(int64_t n) {
+    return (((n + TOPK_WARPS - 1) / TOPK_WARPS) + 31) & ~(int64_t)31;
+}
+
+// The emission's placement: with wcnt[w] = (keys above the bucket, keys in
+// the bucket) of warp w's index range [w*span, (w+1)*span), write the keys
+// above the bucket and the first `need` keys of the bucket in ascending index
+// order, then -1 up to `width`.  The bucket is the keys whose order key under
+// `mask` equals `prefix`.  Called by all TOPK_NT threads.
+__device__ void place_keys(const float* __restrict__ row, int64_t n, int64_t span, uint32_t prefix, uint32_t mask,
+                           uint32_t need, int k, int width, uint32_t (*wcnt)[2], int32_t* __restrict__ out,
+                           StatusHdr* st, int64_t t) {
+    __shared__ uint32_t above_all;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t w0 = (int64_t)warp * span, w1 = min(n, w0 + span);
+    if (warp == 0) {  // exclusive prefixes over the warps, in index order
+        const uint32_t a = wcnt[lane][0], e = wcnt[lane][1];
+        uint32_t ia = a, ie = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t va = __shfl_up_sync(0xffffffffu, ia, o), ve = __shfl_up_sync(0xffffffffu, ie, o);
+            if (lane >= o) ia += va, ie += ve;
+        }
+        wcnt[lane][0] = ia - a;
+        wcnt[lane][1] = ie - e;
+        if (lane == 31) above_all = ia;  // keys above the bucket in all
+    }
+    __syncthreads();
+    uint32_t eq_before = wcnt[warp][1];
+    uint32_t pos = wcnt[warp][0] + min(eq_before, need);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t s0 = w0; s0 < w1; s0 += 32 * TOPK_BATCH) {
+        uint32_t mk[TOPK_BATCH];  // the batch's loads first
+#pragma unroll
+        for (int j = 0; j < TOPK_BATCH; ++j) {
+            const int64_t s = s0 + 32 * j + lane;
+            mk[j] = s < w1 ? (order_key(row[s]) & mask) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < TOPK_BATCH; ++j) {
+            const int64_t s = s0 + 32 * j + lane;
+            const bool ab = s < w1 && mk[j] > prefix, eq = s < w1 && mk[j] == prefix;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool take = ab || (eq && eq_before + (uint32_t)__popc(eqm & lt) < need);
+            const uint32_t tk = __ballot_sync(0xffffffffu, take);
+            if (take && pos + (uint32_t)__popc(tk & lt) < (uint32_t)k) out[pos + __popc(tk & lt)] = (int32_t)s;
+            pos += (uint32_t)__popc(tk);
+            eq_before += (uint32_t)__popc(eqm);
+        }
+    }
+    const uint32_t total = above_all + need;
+    for (int64_t s = total + threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+    if (threadIdx.x == 0 && total != (uint32_t)k) report(st, DSA_ERR_INDEX, -1000000 - t);
+}
+
 __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld,
                                                             int64_t row_begin, int width, const int32_t* __restrict__ k_rows,
                                                             int32_t* __restrict__ idx, int64_t ld_idx, StatusHdr* st) {
@@ -273,9 +454,17 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
         const int shift = 24 - 8 * pass;
         for (int i = threadIdx.x; i < 256; i += TOPK_NT) hist[i] = 0;
         __syncthreads();
-        for (int64_t s = threadIdx.x; s < n; s += TOPK_NT) {
-            const uint32_t key = order_key(row[s]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        for (int64_t s0 = 0; s0 < n; s0 += (int64_t)TOPK_NT * 4) {
+            uint32_t kk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t s = s0 + j * TOPK_NT + threadIdx.x;
+                kk[j] = s < n ? order_key(row[s]) : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (s0 + j * TOPK_NT + threadIdx.x < n && (kk[j] & mask) == prefix)
+                    atomicAdd(&hist[(kk[j] >> shift) & 255u], 1u);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -319,13 +508,22 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
         if (in_bin == need) break;
     }
     // ---- emission: warp w owns indices [w*span, (w+1)*span) ----
-    const int64_t span = (((n + TOPK_WARPS - 1) / TOPK_WARPS) + 31) & ~(int64_t)31;
+    const int64_t span = topk_span(n);
     const int64_t w0 = (int64_t)warp * span, w1 = min(n, w0 + span);
     uint32_t n_above = 0, n_eq = 0;
-    for (int64_t s = w0 + lane; s < w1; s += 32) {
-        const uint32_t m = order_key(row[s]) & mask;
-        n_above += m > prefix;
-        n_eq += m == prefix;
+    for (int64_t s0 = w0; s0 < w1; s0 += 32 * TOPK_BATCH) {
+        uint32_t mk[TOPK_BATCH];
+#pragma unroll
+        for (int j = 0; j < TOPK_BATCH; ++j) {
+            const int64_t s = s0 + 32 * j + lane;
+            mk[j] = s < w1 ? (order_key(row[s]) & mask) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < TOPK_BATCH; ++j) {
+            const bool in = s0 + 32 * j + lane < w1;
+            n_above += in && mk[j] > prefix;
+            n_eq += in && mk[j] == prefix;
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -337,36 +535,282 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
         wcnt[warp][1] = n_eq;
     }
     __syncthreads();
-    if (warp == 0) {  // exclusive prefixes over the warps, in index order
-        const uint32_t a = wcnt[lane][0], e = wcnt[lane][1];
-        uint32_t ia = a, ie = e;
+    place_keys(row, n, span, prefix, mask, need, k, width, wcnt, out, st, t);
+}
+
+// ---------------------------------------------------------------------------
+// a3 for non-negative scores (the selection's own ReLU scores, +inf for NaN):
+// exact top-k of one row per CTA, same result as topk_rows_kernel.
+//   1. A shared-memory histogram of the row over 4096 bins of 1/16 binade
+//      (fp32 bits >> 19).  Zero scores, typically half of a ReLU row, are
+//      counted in 32 per-lane bins and summed after, so they cause no
+//      atomic conflicts.  The bin of the k-th largest score is the bucket.
+//   2. While the bucket holds more than TOPK_CAND keys, a radix pass over the
+//      row refines it by the next digit (bits 18..11, 10..3, 2..0).
+//   3. One pass over the row counts each warp's keys above the bucket and
+//      lists the bucket's keys on chip.
+//   4. The listed keys are refined by the remaining digits in shared memory
+//      until the bucket is one score value or is taken whole.
+//   5. The placement pass writes the keys above the bucket and the first
+//      `need` keys of the bucket in ascending index order.
+// Three passes over the row (L2-resident after the scan) in the usual case.
+// ---------------------------------------------------------------------------
+constexpr int TOPK_CAND = 2048;
+constexpr int TH_BINS = 4096, TH_SHIFT = 19;
+
+// Radix digit `pass` below the 1/16-binade bin: bits 18..11, 10..3, 2..0.
+__device__ __forceinline__ void th_digit(int pass, int& shift, uint32_t& dm) {
+    shift = pass == 0 ? 11 : (pass == 1 ? 3 : 0);
+    dm = pass < 2 ? 0xFFu : 0x7u;
+}
+
+// Warp 0: the bin of a 256-bin digit histogram holding the need-th largest
+// key, the keys above it and its count.
+__device__ __forceinline__ void th_pick(const uint32_t* h, uint32_t need, uint32_t& b_sel, uint32_t& b_above,
+                                        uint32_t& b_count) {
+    const int lane = threadIdx.x & 31;
+    uint32_t cc[8], sm = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t va = __shfl_up_sync(0xffffffffu, ia, o), ve = __shfl_up_sync(0xffffffffu, ie, o);
-            if (lane >= o) ia += va, ie += ve;
+    for (int i = 0; i < 8; ++i) {
+        cc[i] = h[lane * 8 + i];
+        sm += cc[i];
+    }
+    uint32_t in2 = sm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, in2, o);
+        if (lane + o < 32) in2 += v;
+    }
+    const uint32_t ab = in2 - sm;
+    if (ab < need && ab + sm >= need) {
+        uint32_t acc = ab;
+        bool found = false;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            if (!found && acc + cc[i] >= need) {
+                b_sel = (uint32_t)(lane * 8 + i);
+                b_above = acc;
+                b_count = cc[i];
+                found = true;
+            }
+            acc += cc[i];
         }
-        wcnt[lane][0] = ia - a;
-        wcnt[lane][1] = ie - e;
-        if (lane == 31) sel_above = ia;  // keys above the bucket in all
+    }
+}
+
+__global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld,
+                                                            int64_t row_begin, int width, const int32_t* __restrict__ k_rows,
+                                                            int32_t* __restrict__ idx, int64_t ld_idx, StatusHdr* st) {
+    __shared__ __align__(16) uint32_t hb[TH_BINS + 32];
+    __shared__ uint32_t ckey[TOPK_CAND];
+    __shared__ int32_t cidx[TOPK_CAND];
+    __shared__ uint32_t hs[256];
+    __shared__ uint32_t wtot[TOPK_WARPS];
+    __shared__ uint32_t wcnt[TOPK_WARPS][2];
+    __shared__ uint32_t b_sel, b_above, b_count, n_cand;
+    const int64_t r = blockIdx.x;
+    const int64_t t = row_begin + r;
+    const RowInfo ri = row_info(sv, t);
+    int32_t* out = idx + r * ld_idx;
+    if (!ri.ok) {
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, t);
+        return;
+    }
+    const int64_t n = ri.pos + 1;
+    const float* row = scores + r * ld;
+    const int k = k_rows ? min(max(__ldg(k_rows + t), 0), width) : width;
+    if (n <= k || k == 0) {
+        for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = (s < n && s < k) ? (int32_t)s : -1;
+        return;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t need = (uint32_t)k;
+
+    // ---- 1. histogram of the row; the bucket ----
+    for (int i = threadIdx.x; i < TH_BINS + 32; i += TOPK_NT) hb[i] = 0;
+    if (threadIdx.x == 0) b_sel = 0xFFFFFFFFu;
+    __syncthreads();
+    for (int64_t s0 = 0; s0 < n; s0 += (int64_t)TOPK_NT * 4) {
+        uint32_t kk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t s = s0 + j * TOPK_NT + threadIdx.x;
+            kk[j] = s < n ? min(__float_as_uint(row[s]) >> TH_SHIFT, (uint32_t)TH_BINS - 1) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (s0 + j * TOPK_NT + threadIdx.x < n) atomicAdd(&hb[kk[j] ? kk[j] : TH_BINS + lane], 1u);
     }
     __syncthreads();
-    uint32_t eq_before = wcnt[warp][1];
-    uint32_t pos = wcnt[warp][0] + min(eq_before, need);
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t s0 = w0; s0 < w1; s0 += 32) {
-        const int64_t s = s0 + lane;
-        const uint32_t m = s < w1 ? (order_key(row[s]) & mask) : 0u;
-        const bool ab = s < w1 && m > prefix, eq = s < w1 && m == prefix;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-        const bool take = ab || (eq && eq_before + (uint32_t)__popc(eqm & lt) < need);
-        const uint32_t tk = __ballot_sync(0xffffffffu, take);
-        if (take && pos + (uint32_t)__popc(tk & lt) < (uint32_t)k) out[pos + __popc(tk & lt)] = (int32_t)s;
-        pos += (uint32_t)__popc(tk);
-        eq_before += (uint32_t)__popc(eqm);
+    if (warp == 0) {  // bin 0 = the per-lane zero bins
+        uint32_t z = hb[TH_BINS + lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (lane == 0) hb[0] = z;
     }
-    const uint32_t total = sel_above + need;
-    for (int64_t s = total + threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
-    if (threadIdx.x == 0 && total != (uint32_t)k) report(st, DSA_ERR_INDEX, -1000000 - t);
+    __syncthreads();
+    static_assert(TH_BINS == 4 * TOPK_NT, "four bins per thread");
+    const uint4 c4 = *(const uint4*)(hb + 4 * threadIdx.x);
+    const uint32_t c[4] = {c4.x, c4.y, c4.z, c4.w};
+    const uint32_t sum = c[0] + c[1] + c[2] + c[3];
+    uint32_t inc = sum;  // bins of this lane and the lanes above it, in this warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, inc, o);
+        if (lane + o < 32) inc += v;
+    }
+    if (lane == 0) wtot[warp] = inc;
+    __syncthreads();
+    uint32_t above = inc - sum;
+    for (int w = warp + 1; w < TOPK_WARPS; ++w) above += wtot[w];
+    if (above < need && above + sum >= need) {
+        uint32_t acc = above;
+        bool found = false;
+#pragma unroll
+        for (int i = 3; i >= 0; --i) {
+            if (!found && acc + c[i] >= need) {
+                b_sel = 4 * threadIdx.x + i;
+                b_above = acc;
+                b_count = c[i];
+                found = true;
+            }
+            acc += c[i];
+        }
+    }
+    __syncthreads();
+    if (b_sel == 0xFFFFFFFFu) {  // cannot happen with n > k keys counted; reported
+        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, -4000000 - t);
+        for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+        return;
+    }
+    // the bucket in order-key space (non-negative scores: key = bits | 2^31)
+    uint32_t prefix = 0x80000000u | (b_sel << TH_SHIFT);
+    uint32_t mask = 0xFFFFFFFFu << TH_SHIFT;
+    need -= b_above;
+    uint32_t cnt = b_count;
+
+    // ---- 2. refine an oversized bucket by radix passes over the row ----
+    int lvl = 0;
+    for (; lvl < 3 && cnt > (uint32_t)TOPK_CAND && cnt != need; ++lvl) {
+        int shift;
+        uint32_t dm;
+        th_digit(lvl, shift, dm);
+        for (int i = threadIdx.x; i < 256; i += TOPK_NT) hs[i] = 0;
+        __syncthreads();
+        for (int64_t s0 = 0; s0 < n; s0 += (int64_t)TOPK_NT * 4) {
+            uint32_t kk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t s = s0 + j * TOPK_NT + threadIdx.x;
+                kk[j] = s < n ? order_key(row[s]) : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (s0 + j * TOPK_NT + threadIdx.x < n && (kk[j] & mask) == prefix)
+                    atomicAdd(&hs[(kk[j] >> shift) & dm], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) th_pick(hs, need, b_sel, b_above, b_count);
+        __syncthreads();
+        prefix |= b_sel << shift;
+        mask |= dm << shift;
+        need -= b_above;
+        cnt = b_count;
+        __syncthreads();
+    }
+    const bool listed = cnt <= (uint32_t)TOPK_CAND && cnt != need;  // else the bucket is taken whole or is one value
+
+    // ---- 3. per warp: keys above the bucket, keys in it; list the bucket ----
+    const int64_t span = topk_span(n);
+    const int64_t w0 = (int64_t)warp * span, w1 = min(n, w0 + span);
+    if (threadIdx.x == 0) n_cand = 0;
+    __syncthreads();
+    uint32_t n_ab = 0, n_eq = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t s00 = w0; s00 < w1; s00 += 32 * TOPK_BATCH) {
+        uint32_t kb[TOPK_BATCH];
+#pragma unroll
+        for (int j = 0; j < TOPK_BATCH; ++j) {
+            const int64_t s = s00 + 32 * j + lane;
+            kb[j] = s < w1 ? order_key(row[s]) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < TOPK_BATCH; ++j) {
+            const int64_t s = s00 + 32 * j + lane;
+            const uint32_t key = kb[j];
+            const bool ab = s < w1 && (key & mask) > prefix, eq = s < w1 && (key & mask) == prefix;
+            n_ab += ab;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            n_eq += (uint32_t)__popc(eqm) * (lane == 0);
+            if (listed && eqm) {
+                uint32_t base = 0;
+                if (lane == 0) base = atomicAdd(&n_cand, (uint32_t)__popc(eqm));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const uint32_t slot = base + (uint32_t)__popc(eqm & lt);
+                if (eq && slot < (uint32_t)TOPK_CAND) {
+                    ckey[slot] = key;
+                    cidx[slot] = (int32_t)s;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n_ab += __shfl_xor_sync(0xffffffffu, n_ab, o);
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
+    if (lane == 0) {
+        wcnt[warp][0] = n_ab;
+        wcnt[warp][1] = n_eq;
+    }
+    __syncthreads();
+
+    // ---- 4. refine the listed bucket on chip ----
+    if (listed) {
+        const uint32_t nc = n_cand;
+        if (nc != cnt) {  // the row changed under the passes: reported, no indices
+            if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, -5000000 - t);
+            for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+            return;
+        }
+        for (; lvl < 3 && cnt != need; ++lvl) {
+            int shift;
+            uint32_t dm;
+            th_digit(lvl, shift, dm);
+            for (int i = threadIdx.x; i < 256; i += TOPK_NT) hs[i] = 0;
+            __syncthreads();
+            for (uint32_t i = threadIdx.x; i < nc; i += TOPK_NT) {
+                const uint32_t key = ckey[i];
+                if ((key & mask) == prefix) atomicAdd(&hs[(key >> shift) & dm], 1u);
+            }
+            __syncthreads();
+            if (warp == 0) th_pick(hs, need, b_sel, b_above, b_count);
+            __syncthreads();
+            prefix |= b_sel << shift;
+            mask |= dm << shift;
+            need -= b_above;
+            cnt = b_count;
+            __syncthreads();
+        }
+        // per warp: listed keys above the refined bucket, and in it
+        if (threadIdx.x < TOPK_WARPS) wcnt[threadIdx.x][1] = 0;
+        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < nc; i += TOPK_NT) {
+            const uint32_t km = ckey[i] & mask;
+            const int w = (int)(cidx[i] / span);
+            if (km > prefix) atomicAdd(&wcnt[w][0], 1u);
+            else if (km == prefix) atomicAdd(&wcnt[w][1], 1u);
+        }
+        __syncthreads();
+    }
+    // ---- 5. placement ----
+    place_keys(row, n, span, prefix, mask, need, k, width, wcnt, out, st, t);
+}
+
+void launch_topk_hist(const TopkArgs& a, cudaStream_t s) {
+    if (a.row_count <= 0) return;
+    topk_hist_kernel<<<(unsigned)a.row_count, TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k, a.k_rows, a.idx,
+                                                              a.ld_idx, a.st);
 }
 
 void launch_topk_rows(const TopkArgs& a, cudaStream_t s) {

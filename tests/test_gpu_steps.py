@@ -24,9 +24,11 @@ def _fp8_decode(ctx, name="decode_small"):
 
 
 # ---------------------------------------------------------------- a1 fold
-@pytest.mark.parametrize("wl", ["tiny_l512", "fp8_1000"])
+@pytest.mark.parametrize("wl", ["tiny_l512", "fp8_1000", "fp8_3000", "fp8_20000"])
 def test_fold(wl):
-    wl = W.WORKLOADS["tiny_l512"] if wl == "tiny_l512" else _fp8_prefill(1000)
+    # 1000 rows: a column of W per thread; 3000: 2 rows per warp; 20000: 8 rows
+    # per warp on persistent CTAs, ragged last group
+    wl = W.WORKLOADS["tiny_l512"] if wl == "tiny_l512" else _fp8_prefill(int(wl[4:]))
     inp, prob = make(wl)
     u, s = gpu_fold(prob)
     uo, so = oracle.fold(inp.q_idx, inp.q_idx_scale, inp.W)
