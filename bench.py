@@ -679,7 +679,7 @@ def native(args):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": byts / (datt_max / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_launch": byts},
             "select_hbm": {"bytes_scan": scan_bytes, "achieved_gbs": scan_bytes / (dsel / 1e3) / 1e9},
-            "gpu_launches": 5 * dsteps,
+            "gpu_launches": 4 * dsteps,  # fold, scan, top-k, attention
         }
         if not args.no_e2e:
             e2e_ms, h2d, d2h = e2e_native(dinp, dprob, 5)

@@ -14,7 +14,7 @@ under the zigzag, balanced and contiguous plans:
   * context_parallel.forward at world size 1 (the gather's local path and
     both zigzag chunks) equals it as well;
   * a short chunk at the end of the sequence (42 queries over 8192 keys),
-    which takes the scan + radix top-k selection path, agrees in its
+    which takes the scan + histogram top-k selection path, agrees in its
     selection (overlap >= 0.999).  Where its index rows are identical, the
     attention output is identical.
 """

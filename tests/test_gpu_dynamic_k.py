@@ -6,8 +6,8 @@ three selection paths, with per-query k drawn uniformly in [0, k] plus the
 edge values 0, 1, k and past k:
   * prefill_l32768: the fused tensor-core indexer / top-k;
   * prefill_l8192: 64 row blocks over 8192 keys, which selects in two
-    launches (split tensor-core score sweep, then the radix top-k);
-  * decode_b64: the scan + radix top-k.
+    launches (split tensor-core score sweep, then the histogram top-k);
+  * decode_b64: the scan + the histogram top-k.
 Each is checked as follows:
   * the fused selection equals, bit for bit, the exact top-K_t of the GPU's
     own scores (dsa_index_scores ranked by the oracle's top-k), in ascending

@@ -3,8 +3,8 @@
 The selection runs fused (one tensor-core indexer / top-k kernel) at 32K and
 128K and on the batched case (sequences of at most 2048 keys).  prefill_l8192
 and the 3000-token case (fewer 128-row blocks than SMs over more than 2048
-keys) take the two-launch path: a key-split score sweep, then the radix
-top-k.
+keys) take the two-launch path: a key-split score sweep, then the
+histogram top-k.
 For every checked row: the selection equals dsa_topk applied to the
 scores of dsa_index_scores (same arithmetic, bit-exact), its overlap with
 the oracle's own selection is >= 0.999, and the attention output matches the
@@ -104,7 +104,7 @@ def test_forward_tiny_l512():
 
 
 def test_forward_small_prefill_selection_heavy():
-    """k much smaller than L: every row block runs the radix sweeps."""
+    """k much smaller than L: every row's k-th score is deep in its tail."""
     wl = W.custom("prefill_l3000_k256", (3000,), (3000,), base="prefill_l8192", k=256)
     _run(wl, 3000, 48, [(0, 3000)])
 
