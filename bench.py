@@ -64,10 +64,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
     ap.add_argument("--probe-fp8-peak", action="store_true",
                     help="only measure the dense FP8 (e4m3) GEMM peak of this GPU (burst and sustained) and print it")
-    ap.add_argument("--profile-case", choices=["select", "decode-small"],
+    ap.add_argument("--profile-case", choices=["select", "decode-small", "decode"],
                     help="run a lean case for a profiler (no timing line): 'select' = dsa_select on --workload with "
                          "the indexer inputs only; 'decode-small' = decode select + attention, 64 sequences with "
-                         "contexts 16K-24K")
+                         "contexts 16K-24K; 'decode' = the same on decode_b64 (contexts 16K-64K)")
     ap.add_argument("--reps", type=int, default=3, help="calls of the --profile-case")
     return ap.parse_args()
 
@@ -770,9 +770,12 @@ def profile_case(args):
         torch.cuda.synchronize()
         dsa.check_device_status(ws, "profile case select")
     else:
-        rng = np.random.default_rng(0)
-        ctx = tuple(int(x) for x in rng.integers(16384, 24577, size=64))
-        wl = W.custom("decode_b64_ctx16k_24k", (1,) * 64, ctx, base="decode_b64")
+        if args.profile_case == "decode":
+            wl = W.WORKLOADS["decode_b64"]
+        else:
+            rng = np.random.default_rng(0)
+            ctx = tuple(int(x) for x in rng.integers(16384, 24577, size=64))
+            wl = W.custom("decode_b64_ctx16k_24k", (1,) * 64, ctx, base="decode_b64")
         prob = DeviceProblem(W.generate(wl, device="cuda"))
         for _ in range(args.reps):
             dsa.dsa_select(prob.seqs, prob.ia, wl.k, prob.idx, prob.ws)

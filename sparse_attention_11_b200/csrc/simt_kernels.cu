@@ -264,7 +264,10 @@ __global__ void __launch_bounds__(128) scores_f32_kernel(SeqView sv, const float
 // FMA of the exact e4m3 products, xor-shuffle reduction; score =
 // ReLU((dot * s_k) * s_row).  HBM-bound: 132 bytes read per key.
 // ---------------------------------------------------------------------------
-constexpr int SCAN_KEYS = 1024;
+#ifndef DSA_SCAN_KEYS
+#define DSA_SCAN_KEYS 1024
+#endif
+constexpr int SCAN_KEYS = DSA_SCAN_KEYS;
 
 // 16 e4m3 codes (one 16-byte slice of a key) dotted with 16 fp32 query
 // values: the codes are decoded in pairs by the hardware conversion to f16
@@ -285,7 +288,10 @@ __device__ __forceinline__ float dot16_e4m3(const float (&uq)[16], uint4 v) {
     return acc;
 }
 
-constexpr int SCAN_UNROLL = 4;  // keys per lane group in flight
+#ifndef DSA_SCAN_UNROLL
+#define DSA_SCAN_UNROLL 4
+#endif
+constexpr int SCAN_UNROLL = DSA_SCAN_UNROLL;  // keys per lane group in flight
 
 __global__ void __launch_bounds__(256) scan_fp8_kernel(SeqView sv, const uint8_t* __restrict__ u8,
                                                        const float* __restrict__ s_row, const uint8_t* __restrict__ k8,
@@ -540,23 +546,43 @@ __global__ void __launch_bounds__(TOPK_NT) topk_rows_kernel(SeqView sv, const fl
 
 // ---------------------------------------------------------------------------
 // a3 for non-negative scores (the selection's own ReLU scores, +inf for NaN):
-// exact top-k of one row per CTA, same result as topk_rows_kernel.
-//   1. A shared-memory histogram of the row over 4096 bins of 1/16 binade
-//      (fp32 bits >> 19).  Zero scores, typically half of a ReLU row, are
-//      counted in 32 per-lane bins and summed after, so they cause no
-//      atomic conflicts.  The bin of the k-th largest score is the bucket.
-//   2. While the bucket holds more than TOPK_CAND keys, a radix pass over the
-//      row refines it by the next digit (bits 18..11, 10..3, 2..0).
-//   3. One pass over the row counts each warp's keys above the bucket and
-//      lists the bucket's keys on chip.
-//   4. The listed keys are refined by the remaining digits in shared memory
-//      until the bucket is one score value or is taken whole.
-//   5. The placement pass writes the keys above the bucket and the first
-//      `need` keys of the bucket in ascending index order.
+// exact top-k of one row, same result as topk_rows_kernel.  A row is split
+// over a cluster of CPR CTAs (contiguous index ranges, 32 warps each), which
+// merge their counts through distributed shared memory:
+//   1. Each CTA histograms its range over 4096 bins of 1/16 binade (fp32
+//      bits >> 19); zero scores, typically half of a ReLU row, go to 32
+//      per-lane bins summed afterwards, so they cause no atomic conflicts.
+//      Every CTA sums the cluster's histograms and finds the same bucket:
+//      the bin of the k-th largest score.
+//   2. While the bucket holds more than TOPK_CAND keys, radix passes over the
+//      row refine it by the next digit (bits 18..11, 10..3, 2..0).
+//   3. One pass counts each warp's keys above and in the bucket and lists the
+//      bucket's keys in the CTA's shared memory.
+//   4. Every CTA refines the bucket by the remaining digits over all the
+//      cluster's lists, until it is one score value or is taken whole.
+//   5. The CTAs exchange their counts and place their keys: those above the
+//      bucket and the first `need` of the bucket, in ascending index order.
 // Three passes over the row (L2-resident after the scan) in the usual case.
 // ---------------------------------------------------------------------------
 constexpr int TOPK_CAND = 2048;
 constexpr int TH_BINS = 4096, TH_SHIFT = 19;
+
+DSA_DEV uint32_t ld_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+DSA_DEV uint4 ld_cluster_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+DSA_DEV void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // Radix digit `pass` below the 1/16-binade bin: bits 18..11, 10..3, 2..0.
 __device__ __forceinline__ void th_digit(int pass, int& shift, uint32_t& dm) {
@@ -598,48 +624,64 @@ __device__ __forceinline__ void th_pick(const uint32_t* h, uint32_t need, uint32
     }
 }
 
-__global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld,
-                                                            int64_t row_begin, int width, const int32_t* __restrict__ k_rows,
-                                                            int32_t* __restrict__ idx, int64_t ld_idx, StatusHdr* st) {
+template <int CPR>
+__global__ void __cluster_dims__(CPR, 1, 1) __launch_bounds__(TOPK_NT, 2)
+    topk_hist_kernel(SeqView sv, const float* __restrict__ scores, int64_t ld, int64_t row_begin, int width,
+                     const int32_t* __restrict__ k_rows, int32_t* __restrict__ idx, int64_t ld_idx, StatusHdr* st) {
     __shared__ __align__(16) uint32_t hb[TH_BINS + 32];
     __shared__ uint32_t ckey[TOPK_CAND];
     __shared__ int32_t cidx[TOPK_CAND];
-    __shared__ uint32_t hs[256];
+    __shared__ uint32_t hs[256], hsum[256];
     __shared__ uint32_t wtot[TOPK_WARPS];
     __shared__ uint32_t wcnt[TOPK_WARPS][2];
+    __shared__ uint32_t ctot[CPR][2];
     __shared__ uint32_t b_sel, b_above, b_count, n_cand;
-    const int64_t r = blockIdx.x;
+    const uint32_t crank = CPR > 1 ? cluster_ctarank() : 0u;
+    const int64_t r = blockIdx.x / CPR;
     const int64_t t = row_begin + r;
     const RowInfo ri = row_info(sv, t);
     int32_t* out = idx + r * ld_idx;
+    // every decision below is the same in all CTAs of the cluster (same row,
+    // same merged counts), so the cluster leaves or syncs together
     if (!ri.ok) {
-        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, t);
+        if (threadIdx.x == 0 && crank == 0) report(st, DSA_ERR_INDEX, t);
         return;
     }
-    const int64_t n = ri.pos + 1;
+    const int n = (int)(ri.pos + 1);  // index rows are int32: a row has fewer than 2^31 keys
     const float* row = scores + r * ld;
     const int k = k_rows ? min(max(__ldg(k_rows + t), 0), width) : width;
     if (n <= k || k == 0) {
-        for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = (s < n && s < k) ? (int32_t)s : -1;
+        if (crank == 0)
+            for (int s = threadIdx.x; s < width; s += TOPK_NT) out[s] = (s < n && s < k) ? s : -1;
         return;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int TB = CPR > 1 ? TOPK_BATCH : 4;  // keys per lane loaded ahead (registers: two CTAs per SM)
     uint32_t need = (uint32_t)k;
+    // warp g = crank * 32 + warp of the cluster owns [g * span, (g + 1) * span)
+    const int span = (((n + CPR * TOPK_WARPS - 1) / (CPR * TOPK_WARPS)) + 31) & ~31;
+    const int c0 = min(n, (int)crank * TOPK_WARPS * span), c1 = min(n, c0 + TOPK_WARPS * span);
+    auto leave = [&](int code) {  // reported once; no indices; the cluster leaves together
+        if (threadIdx.x == 0 && crank == 0) report(st, DSA_ERR_INDEX, code - t);
+        if (crank == 0)
+            for (int s = threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+        if constexpr (CPR > 1) cluster_sync();
+    };
 
-    // ---- 1. histogram of the row; the bucket ----
+    // ---- 1. histogram of this CTA's range; the cluster's bucket ----
     for (int i = threadIdx.x; i < TH_BINS + 32; i += TOPK_NT) hb[i] = 0;
     if (threadIdx.x == 0) b_sel = 0xFFFFFFFFu;
     __syncthreads();
-    for (int64_t s0 = 0; s0 < n; s0 += (int64_t)TOPK_NT * 4) {
+    for (int s0 = c0; s0 < c1; s0 += TOPK_NT * 4) {
         uint32_t kk[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int64_t s = s0 + j * TOPK_NT + threadIdx.x;
-            kk[j] = s < n ? min(__float_as_uint(row[s]) >> TH_SHIFT, (uint32_t)TH_BINS - 1) : 0u;
+            const int s = s0 + j * TOPK_NT + (int)threadIdx.x;
+            kk[j] = s < c1 ? min(__float_as_uint(row[s]) >> TH_SHIFT, (uint32_t)TH_BINS - 1) : 0u;
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            if (s0 + j * TOPK_NT + threadIdx.x < n) atomicAdd(&hb[kk[j] ? kk[j] : TH_BINS + lane], 1u);
+            if (s0 + j * TOPK_NT + (int)threadIdx.x < c1) atomicAdd(&hb[kk[j] ? kk[j] : TH_BINS + lane], 1u);
     }
     __syncthreads();
     if (warp == 0) {  // bin 0 = the per-lane zero bins
@@ -650,8 +692,20 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
     }
     __syncthreads();
     static_assert(TH_BINS == 4 * TOPK_NT, "four bins per thread");
-    const uint4 c4 = *(const uint4*)(hb + 4 * threadIdx.x);
-    const uint32_t c[4] = {c4.x, c4.y, c4.z, c4.w};
+    uint32_t c[4];
+    if constexpr (CPR > 1) {
+        cluster_sync();  // every CTA's histogram is complete
+        c[0] = c[1] = c[2] = c[3] = 0;
+        const uint32_t my = smem_u32(hb + 4 * threadIdx.x);
+#pragma unroll
+        for (int q = 0; q < CPR; ++q) {
+            const uint4 v = ld_cluster_v4(mapa(my, (uint32_t)q));
+            c[0] += v.x, c[1] += v.y, c[2] += v.z, c[3] += v.w;
+        }
+    } else {
+        const uint4 v = *(const uint4*)(hb + 4 * threadIdx.x);
+        c[0] = v.x, c[1] = v.y, c[2] = v.z, c[3] = v.w;
+    }
     const uint32_t sum = c[0] + c[1] + c[2] + c[3];
     uint32_t inc = sum;  // bins of this lane and the lanes above it, in this warp
 #pragma unroll
@@ -678,9 +732,8 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
         }
     }
     __syncthreads();
-    if (b_sel == 0xFFFFFFFFu) {  // cannot happen with n > k keys counted; reported
-        if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, -4000000 - t);
-        for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+    if (b_sel == 0xFFFFFFFFu) {  // cannot happen with n > k keys counted
+        leave(-4000000);
         return;
     }
     // the bucket in order-key space (non-negative scores: key = bits | 2^31)
@@ -697,46 +750,59 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
         th_digit(lvl, shift, dm);
         for (int i = threadIdx.x; i < 256; i += TOPK_NT) hs[i] = 0;
         __syncthreads();
-        for (int64_t s0 = 0; s0 < n; s0 += (int64_t)TOPK_NT * 4) {
+        for (int s0 = c0; s0 < c1; s0 += TOPK_NT * 4) {
             uint32_t kk[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int64_t s = s0 + j * TOPK_NT + threadIdx.x;
-                kk[j] = s < n ? order_key(row[s]) : 0u;
+                const int s = s0 + j * TOPK_NT + (int)threadIdx.x;
+                kk[j] = s < c1 ? order_key(row[s]) : 0u;
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                if (s0 + j * TOPK_NT + threadIdx.x < n && (kk[j] & mask) == prefix)
+                if (s0 + j * TOPK_NT + (int)threadIdx.x < c1 && (kk[j] & mask) == prefix)
                     atomicAdd(&hs[(kk[j] >> shift) & dm], 1u);
         }
         __syncthreads();
-        if (warp == 0) th_pick(hs, need, b_sel, b_above, b_count);
+        if constexpr (CPR > 1) {
+            cluster_sync();
+            if (threadIdx.x < 256) {
+                uint32_t v = 0;
+                const uint32_t my = smem_u32(hs + threadIdx.x);
+#pragma unroll
+                for (int q = 0; q < CPR; ++q) v += ld_cluster_u32(mapa(my, (uint32_t)q));
+                hsum[threadIdx.x] = v;
+            }
+            __syncthreads();
+            if (warp == 0) th_pick(hsum, need, b_sel, b_above, b_count);
+        } else {
+            if (warp == 0) th_pick(hs, need, b_sel, b_above, b_count);
+        }
         __syncthreads();
         prefix |= b_sel << shift;
         mask |= dm << shift;
         need -= b_above;
         cnt = b_count;
-        __syncthreads();
+        if constexpr (CPR > 1) cluster_sync();  // the cluster's reads of hs are done
+        else __syncthreads();
     }
     const bool listed = cnt <= (uint32_t)TOPK_CAND && cnt != need;  // else the bucket is taken whole or is one value
 
     // ---- 3. per warp: keys above the bucket, keys in it; list the bucket ----
-    const int64_t span = topk_span(n);
-    const int64_t w0 = (int64_t)warp * span, w1 = min(n, w0 + span);
+    const int w0 = min(c1, c0 + warp * span), w1 = min(c1, w0 + span);
     if (threadIdx.x == 0) n_cand = 0;
     __syncthreads();
     uint32_t n_ab = 0, n_eq = 0;
     const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t s00 = w0; s00 < w1; s00 += 32 * TOPK_BATCH) {
-        uint32_t kb[TOPK_BATCH];
+    for (int s00 = w0; s00 < w1; s00 += 32 * TB) {
+        uint32_t kb[TB];
 #pragma unroll
-        for (int j = 0; j < TOPK_BATCH; ++j) {
-            const int64_t s = s00 + 32 * j + lane;
+        for (int j = 0; j < TB; ++j) {
+            const int s = s00 + 32 * j + lane;
             kb[j] = s < w1 ? order_key(row[s]) : 0u;
         }
 #pragma unroll
-        for (int j = 0; j < TOPK_BATCH; ++j) {
-            const int64_t s = s00 + 32 * j + lane;
+        for (int j = 0; j < TB; ++j) {
+            const int s = s00 + 32 * j + lane;
             const uint32_t key = kb[j];
             const bool ab = s < w1 && (key & mask) > prefix, eq = s < w1 && (key & mask) == prefix;
             n_ab += ab;
@@ -749,7 +815,7 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
                 const uint32_t slot = base + (uint32_t)__popc(eqm & lt);
                 if (eq && slot < (uint32_t)TOPK_CAND) {
                     ckey[slot] = key;
-                    cidx[slot] = (int32_t)s;
+                    cidx[slot] = s;
                 }
             }
         }
@@ -764,13 +830,18 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
         wcnt[warp][1] = n_eq;
     }
     __syncthreads();
+    if constexpr (CPR > 1) cluster_sync();  // every CTA's list is complete
 
-    // ---- 4. refine the listed bucket on chip ----
+    // ---- 4. refine the listed bucket over the cluster's lists ----
     if (listed) {
-        const uint32_t nc = n_cand;
-        if (nc != cnt) {  // the row changed under the passes: reported, no indices
-            if (threadIdx.x == 0) report(st, DSA_ERR_INDEX, -5000000 - t);
-            for (int64_t s = threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+        uint32_t nq[CPR], nc = 0;
+#pragma unroll
+        for (int q = 0; q < CPR; ++q) {
+            nq[q] = CPR > 1 ? ld_cluster_u32(mapa(smem_u32(&n_cand), (uint32_t)q)) : n_cand;
+            nc += nq[q];
+        }
+        if (nc != cnt) {  // the row changed under the passes
+            leave(-5000000);
             return;
         }
         for (; lvl < 3 && cnt != need; ++lvl) {
@@ -779,9 +850,14 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
             th_digit(lvl, shift, dm);
             for (int i = threadIdx.x; i < 256; i += TOPK_NT) hs[i] = 0;
             __syncthreads();
-            for (uint32_t i = threadIdx.x; i < nc; i += TOPK_NT) {
-                const uint32_t key = ckey[i];
-                if ((key & mask) == prefix) atomicAdd(&hs[(key >> shift) & dm], 1u);
+#pragma unroll
+            for (int q = 0; q < CPR; ++q) {
+                const uint32_t base = smem_u32(ckey);
+                const uint32_t rb = CPR > 1 ? mapa(base, (uint32_t)q) : base;
+                for (uint32_t i = threadIdx.x; i < nq[q]; i += TOPK_NT) {
+                    const uint32_t key = CPR > 1 ? ld_cluster_u32(rb + 4 * i) : ckey[i];
+                    if ((key & mask) == prefix) atomicAdd(&hs[(key >> shift) & dm], 1u);
+                }
             }
             __syncthreads();
             if (warp == 0) th_pick(hs, need, b_sel, b_above, b_count);
@@ -792,25 +868,87 @@ __global__ void __launch_bounds__(TOPK_NT, 2) topk_hist_kernel(SeqView sv, const
             cnt = b_count;
             __syncthreads();
         }
-        // per warp: listed keys above the refined bucket, and in it
+        // per warp: this CTA's listed keys above the refined bucket, and in it
         if (threadIdx.x < TOPK_WARPS) wcnt[threadIdx.x][1] = 0;
         __syncthreads();
-        for (uint32_t i = threadIdx.x; i < nc; i += TOPK_NT) {
+        for (uint32_t i = threadIdx.x; i < n_cand; i += TOPK_NT) {
             const uint32_t km = ckey[i] & mask;
-            const int w = (int)(cidx[i] / span);
+            const int w = (cidx[i] - c0) / span;
             if (km > prefix) atomicAdd(&wcnt[w][0], 1u);
             else if (km == prefix) atomicAdd(&wcnt[w][1], 1u);
         }
         __syncthreads();
     }
-    // ---- 5. placement ----
-    place_keys(row, n, span, prefix, mask, need, k, width, wcnt, out, st, t);
+
+    // ---- 5. offsets over the warps and the cluster's CTAs; placement ----
+    if (warp == 0) {  // exclusive prefixes over this CTA's warps, in index order
+        const uint32_t a = wcnt[lane][0], e = wcnt[lane][1];
+        uint32_t ia = a, ie = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t va = __shfl_up_sync(0xffffffffu, ia, o), ve = __shfl_up_sync(0xffffffffu, ie, o);
+            if (lane >= o) ia += va, ie += ve;
+        }
+        wcnt[lane][0] = ia - a;
+        wcnt[lane][1] = ie - e;
+        if (lane == 31) {  // this CTA's totals, to every CTA of the cluster
+            if constexpr (CPR > 1) {
+#pragma unroll
+                for (int q = 0; q < CPR; ++q) {
+                    st_cluster_u32(mapa(smem_u32(&ctot[crank][0]), (uint32_t)q), ia);
+                    st_cluster_u32(mapa(smem_u32(&ctot[crank][1]), (uint32_t)q), ie);
+                }
+            } else {
+                ctot[0][0] = ia;
+                ctot[0][1] = ie;
+            }
+        }
+    }
+    if constexpr (CPR > 1) cluster_sync();  // the last access to another CTA's shared memory
+    else __syncthreads();
+    uint32_t base_ab = 0, base_eq = 0, all_ab = 0;
+#pragma unroll
+    for (int q = 0; q < CPR; ++q) {
+        if (q < (int)crank) base_ab += ctot[q][0], base_eq += ctot[q][1];
+        all_ab += ctot[q][0];
+    }
+    uint32_t eq_before = base_eq + wcnt[warp][1];
+    uint32_t pos = base_ab + wcnt[warp][0] + min(eq_before, need);
+    for (int s0 = w0; s0 < w1; s0 += 32 * TB) {
+        uint32_t mk[TB];  // the batch's loads first
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+            const int s = s0 + 32 * j + lane;
+            mk[j] = s < w1 ? (order_key(row[s]) & mask) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+            const int s = s0 + 32 * j + lane;
+            const bool ab = s < w1 && mk[j] > prefix, eq = s < w1 && mk[j] == prefix;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool take = ab || (eq && eq_before + (uint32_t)__popc(eqm & lt) < need);
+            const uint32_t tk = __ballot_sync(0xffffffffu, take);
+            if (take && pos + (uint32_t)__popc(tk & lt) < (uint32_t)k) out[pos + __popc(tk & lt)] = s;
+            pos += (uint32_t)__popc(tk);
+            eq_before += (uint32_t)__popc(eqm);
+        }
+    }
+    const uint32_t total = all_ab + need;
+    if (crank == 0) {
+        for (int s = (int)total + (int)threadIdx.x; s < width; s += TOPK_NT) out[s] = -1;
+        if (threadIdx.x == 0 && total != (uint32_t)k) report(st, DSA_ERR_INDEX, -1000000 - t);
+    }
 }
 
 void launch_topk_hist(const TopkArgs& a, cudaStream_t s) {
     if (a.row_count <= 0) return;
-    topk_hist_kernel<<<(unsigned)a.row_count, TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k, a.k_rows, a.idx,
-                                                              a.ld_idx, a.st);
+    // few rows (decode): four CTAs per row, so that every SM of a B200 works
+    if (a.row_count < 2 * 148)
+        topk_hist_kernel<4><<<(unsigned)(4 * a.row_count), TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k,
+                                                                            a.k_rows, a.idx, a.ld_idx, a.st);
+    else
+        topk_hist_kernel<1><<<(unsigned)a.row_count, TOPK_NT, 0, s>>>(a.sv, a.scores, a.ld, a.row_begin, a.k, a.k_rows,
+                                                                     a.idx, a.ld_idx, a.st);
 }
 
 void launch_topk_rows(const TopkArgs& a, cudaStream_t s) {
