@@ -258,10 +258,11 @@ DSA_API int dsa_indexer_kl(const dsa_seqs* seqs, const float* q_idx, int64_t q_s
  * - Prefill-shaped E4M3 problems run one fused tensor-core indexer / top-k
  *   kernel, one CTA per 128 query rows of a sequence, and the scores never
  *   reach memory.
- * - When such a problem has fewer than 148 row blocks (ceil(max_seqlen_q /
+ * - When such a problem has fewer than 80 row blocks (ceil(max_seqlen_q /
  *   128) x batch) over max_seqlen_k > 2048 keys, and the score buffer
  *   (total_q x max_seqlen_k floats) fits in 8 GiB, the selection runs in two
- *   launches instead.  This is the case of a query chunk over a long prefix.
+ *   launches instead: a short prefill (up to about 10K tokens) or a query
+ *   chunk over a long prefix.
  *   The first launch is a score sweep that splits each block's key range over
  *   several CTAs; the second selects per row from the scores (as below for
  *   decode).  The scores pass through the workspace, and the result is the

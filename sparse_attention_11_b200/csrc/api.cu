@@ -74,15 +74,22 @@ bool use_tc_indexer(const dsa_seqs* s, const dsa_indexer_args* ia) {
 }
 
 // The fused indexer/top-k runs one CTA per 128-row block, which covers the
-// sweeps over the block's whole key range.  With few blocks over long key
-// ranges (a query chunk over a long prefix: context-parallel ranks, chunked
-// prefill), most SMs idle and the longest block sets the time.  There the
-// selection runs as two launches instead: a tensor-core score sweep with
-// each block's key tiles split over several CTAs, then the exact radix
-// top-k per row.  Both rank the same scores exactly, so the indices are
-// identical.  The choice depends only on the shapes, so the workspace size
-// agrees with the call.
-constexpr int64_t kSplitMaxBlocks = 148;       // fewer row blocks than SMs (measured crossover on B200)
+// sweeps over the block's whole key range.  With few blocks (a short
+// prefill, or a query chunk over a long prefix: context-parallel ranks,
+// chunked prefill), most SMs idle and the longest block sets the time.
+// There the selection runs as two launches instead: a tensor-core score
+// sweep with each block's key tiles split over several CTAs, then the exact
+// top-k per row from the scores in memory.  Both rank the same scores
+// exactly, so the indices are identical.  Measured on a B200: two launches
+// win up to 64 blocks (8K prefill 0.40 against 0.45 ms; 2048 rows over 32K
+// keys 0.48 against 0.90), break even at 32 blocks over 32K keys, and lose
+// from 96 blocks on (12K prefill 0.79 against 0.49 ms), where the score
+// buffer's traffic grows with rows x keys.  The choice depends only on the
+// shapes, so the workspace size agrees with the call.
+#ifndef DSA_SPLIT_MAX_BLOCKS
+#define DSA_SPLIT_MAX_BLOCKS 80
+#endif
+constexpr int64_t kSplitMaxBlocks = DSA_SPLIT_MAX_BLOCKS;  // two launches below this many row blocks
 constexpr int64_t kSplitMinKeys = 2049;        // key ranges longer than 2048 (shorter ones need few sweeps)
 constexpr size_t kSplitMaxScoreBytes = (size_t)8 << 30;
 

@@ -2,7 +2,7 @@
 
 The selection runs fused (one tensor-core indexer / top-k kernel) at 32K and
 128K and on the batched case (sequences of at most 2048 keys).  prefill_l8192
-and the 3000-token case (fewer 128-row blocks than SMs over more than 2048
+and the 3000-token case (fewer than 80 128-row blocks over more than 2048
 keys) take the two-launch path: a key-split score sweep, then the
 histogram top-k.
 For every checked row: the selection equals dsa_topk applied to the
