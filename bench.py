@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--cp", action="store_true",
                     help="under torchrun: split one sequence over the ranks (context parallel) instead of replicas")
     ap.add_argument("--cp-scheme", choices=["balanced", "zigzag", "contiguous"], default="balanced")
+    ap.add_argument("--kv-reuse", action="store_true",
+                    help="also measure the cross-query KV-tile reuse prototype (adjacent query pairs, k = 1024)")
     ap.add_argument("--bwd", action="store_true",
                     help="also time the sparse attention's backward (dsa_sparse_attn_bwd) on the workload")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU seconds of the oracle sample")
@@ -375,6 +377,84 @@ def dynamic_k_native(inp, prob, steps, warmup, lo=256, seed=11):
             "attention_tflops": flops / (att_ms / 1e3) / 1e12}
 
 
+def kv_reuse_prototype(prob, steps, warmup, k1=1024):
+    """Cross-query KV-tile reuse (adjacent query pairs), a measured prototype
+    on the shipped attention kernel.  Each query of a pair (2i, 2i+1) gets
+    the pair's union of top-k1 selections as its index row (at most 2*k1
+    slots, ascending), with the slots only its partner selected masked (-1):
+    the kernel then runs S, the softmax and PV over the union's tiles with a
+    per-query mask, which is the per-query compute of a kernel that gathers
+    each union tile once for both queries.  A masked slot gathers row 0 (an
+    L2 hit) instead of the partner's key and the tiles after the query's last
+    own slot are skipped, so the time is a lower bound for such a kernel.
+    The baseline is each query over its own k1 keys; outputs must agree
+    (masked slots carry zero weight).  Union sizes give the gather saving."""
+    import numpy as np
+    import torch
+    from sparse_attention_11_b200 import dsa
+    wl = prob.wl
+    T = wl.total_q
+    st = torch.cuda.current_stream()
+    ws = dsa.workspace(dsa.dsa_workspace_size(dsa.DSA_OP_FORWARD, prob.seqs, 2 * k1, prob.ia, prob.aa))
+    own = torch.full((T, k1), -1, dtype=torch.int32, device="cuda")
+    dsa.dsa_select(prob.seqs, prob.ia, k1, own, ws)
+    dsa.check_device_status(ws, "kv reuse: select")
+    npair = T // 2
+    big = torch.iinfo(torch.int64).max
+    a = own[0:2 * npair:2].to(torch.int64)
+    b = own[1:2 * npair:2].to(torch.int64)
+    cat = torch.cat([a, b], dim=1)
+    cat = torch.where(cat < 0, torch.full_like(cat, big), cat)
+    srt, _ = torch.sort(cat, dim=1)
+    dup = torch.zeros_like(srt, dtype=torch.bool)
+    dup[:, 1:] = srt[:, 1:] == srt[:, :-1]
+    uni, _ = torch.sort(torch.where(dup, torch.full_like(srt, big), srt), dim=1)
+    usize = (uni != big).sum(dim=1)
+
+    def masked(rows):
+        o, _ = torch.sort(torch.where(rows < 0, torch.full_like(rows, big), rows), dim=1)
+        j = torch.searchsorted(o, uni).clamp(max=o.shape[1] - 1)
+        hit = (torch.gather(o, 1, j) == uni) & (uni != big)
+        return torch.where(hit, uni, torch.full_like(uni, -1)).to(torch.int32)
+
+    idx_u = torch.full((T, 2 * k1), -1, dtype=torch.int32, device="cuda")
+    idx_u[0:2 * npair:2] = masked(a)
+    idx_u[1:2 * npair:2] = masked(b)
+    if T % 2:
+        idx_u[T - 1, :k1] = own[T - 1]
+    del a, b, cat, srt, dup, uni
+
+    def timed(idx, ksel):
+        for _ in range(warmup):
+            dsa.dsa_sparse_attn(prob.seqs, prob.aa, idx, ksel, ws)
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for e in evs:
+            e[0].record(st)
+            dsa.dsa_sparse_attn(prob.seqs, prob.aa, idx, ksel, ws)
+            e[1].record(st)
+        torch.cuda.synchronize()
+        dsa.check_device_status(ws, "kv reuse: attention")
+        return statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+
+    base_ms = timed(own, k1)
+    out_base = prob.out.clone()
+    lse_base = prob.lse.clone() if prob.lse is not None else None
+    union_ms = timed(idx_u, 2 * k1)
+    diff = float((prob.out.float() - out_base.float()).abs().max())
+    ldiff = float((prob.lse - lse_base).abs().max()) if lse_base is not None else None
+    del out_base, lse_base
+    us = usize.float().cpu().numpy()
+    n_own = int((own >= 0).sum())
+    return {"k_per_query": k1, "pairs": npair, "union_keys_mean": float(us.mean()),
+            "union_keys_p5_p95": [float(np.percentile(us, 5)), float(np.percentile(us, 95))],
+            "attention_ms_own": base_ms, "attention_ms_union_masked": union_ms, "time_ratio": union_ms / base_ms,
+            "gathered_rows_own": n_own, "gathered_rows_shared_tiles": int(usize.sum()) + (k1 if T % 2 else 0),
+            "gather_saving": 1.0 - (int(usize.sum()) + (k1 if T % 2 else 0)) / n_own,
+            "max_abs_diff_out": diff, "max_abs_diff_lse": ldiff,
+            "note": "union tiles with a per-query mask on the shipped kernel: a lower bound of a shared-tile kernel's time"}
+
+
 def context_parallel_emulated(prob, world, schemes, steps, warmup):
     """Context-parallel prefill with its ranks emulated in turn on this GPU.
     Each rank's chunks run against the whole key side, which is what the
@@ -659,6 +739,8 @@ def native(args):
     # dynamic k last: it writes the problem's indices and output with another selection
     if not args.no_dynk and wl.name != "decode_b64":
         res["dynamic_k"] = dynamic_k_native(inp, prob, max(3, min(args.steps, 10)), args.warmup)
+    if args.kv_reuse and wl.batch == 1 and wl.attn_dtype == "bf16":
+        res["kv_reuse_prototype"] = kv_reuse_prototype(prob, max(3, min(args.steps, 10)), args.warmup)
     if not args.no_cp and ws_n == 1 and wl.batch == 1 and wl.idx_dtype == "e4m3":
         res["context_parallel"] = context_parallel_emulated(prob, 8, ("balanced", "zigzag", "contiguous"), 5, 2)
     if not args.no_decode and wl.name != "decode_b64":
