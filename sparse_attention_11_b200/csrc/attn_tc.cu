@@ -43,11 +43,12 @@
 // are free.  A tcgen05.mma takes about 50 cycles to issue from one thread,
 // which makes the 16-20 N=64 MMAs of an S tile issue-bound; so two warps issue
 // an S tile, each half of the contraction blocks into its own accumulator, and
-// the softmax warps add the two.  P tiles are double-buffered and released by a tcgen05.commit that
+// the softmax warps add the two.  P tiles are triple-buffered and released by a tcgen05.commit that
 // arrives on the p_free barrier of both CTAs (PV(t) done in both), so stage B
-// waits for PV(t-2), and for PV(t-1) only when the running maximum moves.
-// The P exchange also keeps the two CTAs within one tile of each other, which
-// the two-arrival p_free barrier relies on.
+// waits for PV(t-3), and for PV(t-1) only when the running maximum moves.
+// The P exchange also keeps the two CTAs' PVs within three tiles of each
+// other (a CTA's half of P(t+3) waits for PV(t) in both), which the
+// two-arrival p_free barrier relies on.
 //
 // Gathers: six producer warps copy the selected rows with 16-byte
 // cp.async, 4 rows x 128 bytes per warp instruction, into the
@@ -118,10 +119,13 @@ struct AtLayout {
     static constexpr uint32_t OFF_INFO = OFF_VM + 512;            // [2][8] last used slot per producer warp, [8] tile counts
     static constexpr uint32_t OFF_BAR = OFF_INFO + 128;
     // epilogue staging: per softmax warp 32 rows x 64 output columns (bf16),
-    // so that the output stores cover whole 128-byte lines
+    // so that the output stores cover whole 128-byte lines; with three P
+    // tiles, 32 rows x 32 columns (64-byte segments) to make room
     static constexpr bool EPI_STAGE = !VSEP && DSA_ATTN_EPI_STAGE;
+    static constexpr int EPI_COLS = NPB >= 3 ? 32 : 64;
+    static constexpr uint32_t EPI_WARP_BYTES = 32 * EPI_COLS * 2;
     static constexpr uint32_t OFF_EPI = OFF_BAR + 512;
-    static constexpr uint32_t SMEM = OFF_EPI + (EPI_STAGE ? 8 * 4096 : 0);
+    static constexpr uint32_t SMEM = OFF_EPI + (EPI_STAGE ? 8 * EPI_WARP_BYTES : 0);
 };
 
 struct AtBars {
@@ -132,8 +136,8 @@ struct AtBars {
     uint64_t q_full;         // Q of the next query with tiles is in place (4 A warps)
     uint64_t o_full;         // all PVs of a query done
     uint64_t o_free;         // its epilogue has read O (8 softmax warps)
-    uint64_t p_full[2];      // 4 local B warps + the peer's half of P (bytes)
-    uint64_t p_free[2];      // PV done in both CTAs (multicast commit)
+    uint64_t p_full[3];      // 4 local B warps + the peer's half of P (bytes)
+    uint64_t p_free[3];      // PV done in both CTAs (multicast commit)
     uint64_t sx_full[2];     // the peer's partial scores (bytes)
     uint64_t sx_free[2];     // the peer consumed the partials this CTA sent
     uint64_t lx_full;        // the peer's row sums (bytes)
@@ -154,7 +158,7 @@ template <int NST, bool VSEP, int NPB, int NSX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ AttnTcArgs a) {
     static_assert(AT_SOFT0 % 4 == 0 && AT_PRODUCERS < AT_SOFT0, "warp roles");
-    static_assert(NST >= 1 && NST <= 4 && NPB >= 1 && NPB <= 2 && NSX >= 1 && NSX <= 2, "barrier arrays");
+    static_assert(NST >= 1 && NST <= 4 && NPB >= 1 && NPB <= 3 && NSX >= 1 && NSX <= 2, "barrier arrays");
     using Lay = AtLayout<NST, VSEP, NPB, NSX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -187,9 +191,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
         mbar_init(smem_u32(&bars->s_empty), 8);  // 4 A + 4 B warps read every S tile
         mbar_init(smem_u32(&bars->s_go), 1);
         mbar_init(smem_u32(&bars->drain2), 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 3; ++i) {
             mbar_init(smem_u32(&bars->p_full[i]), 4);   // (only NPB of them are used)
             mbar_init(smem_u32(&bars->p_free[i]), 2);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&bars->sx_full[i]), 1);
             mbar_init(smem_u32(&bars->sx_free[i]), 4);
             mbar_init(smem_u32(&bars->info_full[i]), AT_PRODUCERS);
@@ -551,11 +557,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(AT_THREADS, 1)
                     w[4 * c + i].z = pack_bf16(__uint_as_float(r[c][8 * i + 4]) * inv, __uint_as_float(r[c][8 * i + 5]) * inv);
                     w[4 * c + i].w = pack_bf16(__uint_as_float(r[c][8 * i + 6]) * inv, __uint_as_float(r[c][8 * i + 7]) * inv);
                 }
-            if constexpr (Lay::EPI_STAGE) {
+            if constexpr (Lay::EPI_STAGE && Lay::EPI_COLS == 32) {
+                // through this warp's staging tile, 32 columns at a time: row =
+                // lane, 16-byte chunk k of the quarter at ((k ^ ((row >> 1) & 3)) << 4);
+                // read back as 8 rows x 64 bytes per instruction
+                uint8_t* stg = smem + Lay::OFF_EPI + (warp - AT_SOFT0) * Lay::EPI_WARP_BYTES;
+                __nv_bfloat16* obase =
+                    a.out + (t - a.row_begin) * a.out_stride_tok + (int64_t)(quad * 32) * a.out_stride_head + dv0 + ocol;
+#pragma unroll
+                for (int qc = 0; qc < 4; ++qc) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        *(uint4*)(stg + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = w[4 * qc + k];
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = 8 * i + (int)(lane >> 2), k = (int)(lane & 3);
+                        const uint4 v = *(const uint4*)(stg + row * 64 + ((k ^ ((row >> 1) & 3)) << 4));
+                        *(uint4*)(obase + (int64_t)row * a.out_stride_head + qc * 32 + k * 8) = v;
+                    }
+                    __syncwarp();
+                }
+            } else if constexpr (Lay::EPI_STAGE) {
                 // through this warp's staging tile: row = lane, 16-byte chunk k of a
                 // 64-column half at ((k ^ (row & 7)) << 4); read back as 4 rows x
                 // 128 bytes per instruction
-                uint8_t* stg = smem + Lay::OFF_EPI + (warp - AT_SOFT0) * 4096;
+                uint8_t* stg = smem + Lay::OFF_EPI + (warp - AT_SOFT0) * Lay::EPI_WARP_BYTES;
                 __nv_bfloat16* obase =
                     a.out + (t - a.row_begin) * a.out_stride_tok + (int64_t)(quad * 32) * a.out_stride_head + dv0 + ocol;
 #pragma unroll
@@ -842,7 +869,7 @@ static bool launch_attn_tc_t(const AttnTcArgs& a, cudaStream_t s) {
 
 #ifndef DSA_ATTN_NST
 #define DSA_ATTN_NST 3
-#define DSA_ATTN_NPB 2
+#define DSA_ATTN_NPB 3
 #define DSA_ATTN_NSX 1
 #endif
 

@@ -32,6 +32,27 @@ def test_select_noalloc_matches_select(L, k):
         assert np.array_equal(out.cpu().numpy(), ref)
 
 
+def test_select_noalloc_ragged_batch_dynamic_k():
+    """A ragged batch of three prefill sequences with a per-query k (k_t
+    uniform in [0, k] plus 0 and past k), against dsa_select."""
+    k = 512
+    wl = W.custom("noalloc_batch", (1500, 700, 2300), (1500, 900, 2300), base="prefill_l8192", k=k)
+    inp = W.generate(wl, device="cuda")
+    prob = DeviceProblem(inp)
+    rng = np.random.default_rng(3)
+    kr = rng.integers(0, k + 1, size=wl.total_q).astype(np.int32)
+    kr[:5] = 0
+    kr[-5:] = k + 100
+    ia = dsa.indexer_args(prob.q_idx, prob.q_idx_scale, prob.W, prob.k_idx, prob.k_idx_scale,
+                          k_per_row=torch.from_numpy(kr).cuda())
+    ref = torch.empty((wl.total_q, k), dtype=torch.int32, device="cuda")
+    dsa.dsa_select(prob.seqs, ia, k, ref, prob.ws)
+    dsa.check_device_status(prob.ws, "dsa_select")
+    out = torch.full((wl.total_q, k), -7, dtype=torch.int32, device="cuda")
+    dsa.dsa_select_noalloc(prob.seqs, ia, k, out)
+    assert np.array_equal(out.cpu().numpy(), ref.cpu().numpy())
+
+
 def test_select_noalloc_rejects_oversize_and_unsupported():
     # more query rows than the static scratch holds: rejected before launch
     L = 32769
