@@ -377,6 +377,40 @@ def dynamic_k_native(inp, prob, steps, warmup, lo=256, seed=11):
             "attention_tflops": flops / (att_ms / 1e3) / 1e12}
 
 
+def pair_union_rows(own):
+    """Index rows for adjacent query pairs (2i, 2i+1) sharing their key
+    tiles: row 2i (2i+1) holds the ascending union of both queries'
+    selections, with the keys only the partner selected set to -1 (masked),
+    then -1 padding, width 2 * own.shape[1].  A trailing unpaired row keeps
+    its own selection.  Returns the rows and the union size of each pair."""
+    import torch
+    T, k1 = own.shape
+    npair = T // 2
+    big = torch.iinfo(torch.int64).max
+    a = own[0:2 * npair:2].to(torch.int64)
+    b = own[1:2 * npair:2].to(torch.int64)
+    cat = torch.cat([a, b], dim=1)
+    cat = torch.where(cat < 0, torch.full_like(cat, big), cat)
+    srt, _ = torch.sort(cat, dim=1)
+    dup = torch.zeros_like(srt, dtype=torch.bool)
+    dup[:, 1:] = srt[:, 1:] == srt[:, :-1]
+    uni, _ = torch.sort(torch.where(dup, torch.full_like(srt, big), srt), dim=1)
+    usize = (uni != big).sum(dim=1)
+
+    def masked(rows):
+        o, _ = torch.sort(torch.where(rows < 0, torch.full_like(rows, big), rows), dim=1)
+        j = torch.searchsorted(o, uni).clamp(max=o.shape[1] - 1)
+        hit = (torch.gather(o, 1, j) == uni) & (uni != big)
+        return torch.where(hit, uni, torch.full_like(uni, -1)).to(torch.int32)
+
+    out = torch.full((T, 2 * k1), -1, dtype=torch.int32, device=own.device)
+    out[0:2 * npair:2] = masked(a)
+    out[1:2 * npair:2] = masked(b)
+    if T % 2:
+        out[T - 1, :k1] = own[T - 1]
+    return out, usize
+
+
 def kv_reuse_prototype(prob, steps, warmup, k1=1024):
     """Cross-query KV-tile reuse (adjacent query pairs), a measured prototype
     on the shipped attention kernel.  Each query of a pair (2i, 2i+1) gets
@@ -400,29 +434,7 @@ def kv_reuse_prototype(prob, steps, warmup, k1=1024):
     dsa.dsa_select(prob.seqs, prob.ia, k1, own, ws)
     dsa.check_device_status(ws, "kv reuse: select")
     npair = T // 2
-    big = torch.iinfo(torch.int64).max
-    a = own[0:2 * npair:2].to(torch.int64)
-    b = own[1:2 * npair:2].to(torch.int64)
-    cat = torch.cat([a, b], dim=1)
-    cat = torch.where(cat < 0, torch.full_like(cat, big), cat)
-    srt, _ = torch.sort(cat, dim=1)
-    dup = torch.zeros_like(srt, dtype=torch.bool)
-    dup[:, 1:] = srt[:, 1:] == srt[:, :-1]
-    uni, _ = torch.sort(torch.where(dup, torch.full_like(srt, big), srt), dim=1)
-    usize = (uni != big).sum(dim=1)
-
-    def masked(rows):
-        o, _ = torch.sort(torch.where(rows < 0, torch.full_like(rows, big), rows), dim=1)
-        j = torch.searchsorted(o, uni).clamp(max=o.shape[1] - 1)
-        hit = (torch.gather(o, 1, j) == uni) & (uni != big)
-        return torch.where(hit, uni, torch.full_like(uni, -1)).to(torch.int32)
-
-    idx_u = torch.full((T, 2 * k1), -1, dtype=torch.int32, device="cuda")
-    idx_u[0:2 * npair:2] = masked(a)
-    idx_u[1:2 * npair:2] = masked(b)
-    if T % 2:
-        idx_u[T - 1, :k1] = own[T - 1]
-    del a, b, cat, srt, dup, uni
+    idx_u, usize = pair_union_rows(own)
 
     def timed(idx, ksel):
         for _ in range(warmup):
