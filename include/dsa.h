@@ -77,8 +77,9 @@ enum dsa_op {
     DSA_OP_FORWARD_HOST = 5
 };
 
-/* Query rows per chunk of dsa_forward_host. */
-#define DSA_HOST_CHUNK_ROWS 2048
+/* Query rows per chunk of dsa_forward_host (the pipeline's fill and drain
+ * are one chunk's copy each, so smaller chunks shorten them). */
+#define DSA_HOST_CHUNK_ROWS 1024
 
 /* Packed variable-length batch (see "Sequences" above). */
 typedef struct dsa_seqs {

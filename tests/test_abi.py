@@ -210,7 +210,7 @@ def test_forward_host_validation(lib):
     fwd = n.value
     assert lib.raw_call("dsa_workspace_size", lib.DSA_OP_FORWARD_HOST, ctypes.byref(S), 2048, ctypes.byref(ia),
                         ctypes.byref(packed), ctypes.byref(n)) == 0
-    chunk = 2048  # DSA_HOST_CHUNK_ROWS
+    chunk = 1024  # DSA_HOST_CHUNK_ROWS
     assert n.value >= fwd + 2 * chunk * h * (dk + dv) * 2
     ws = P(0x10000)
     call = lambda aa, nbytes: lib.raw_call("dsa_forward_host", ctypes.byref(S), ctypes.byref(ia), ctypes.byref(aa),

@@ -158,7 +158,7 @@ def test_fused_selection_matches_oracle_topk_l32768():
 def test_forward_host_matches_forward(name):
     """dsa_forward_host (query and output in pinned host memory, chunked and
     pipelined over three streams) returns exactly dsa_forward's output, lse and
-    indices: 4 chunks at L=8192, 2 chunks for a ragged batch."""
+    indices: 8 chunks at L=8192, 3 chunks for a ragged batch of 2329 rows."""
     wl = W.WORKLOADS[name] if name != "batched" else \
         W.custom("prefill_b3h", (700, 1500, 129), (700, 1500, 129), base="prefill_l8192", k=300)
     inp, prob = make(wl)
