@@ -283,7 +283,7 @@ def step_launches(wl):
     """Kernel launches of one prefill step (dsa_select + dsa_sparse_attn),
     by the library's selection rule (include/dsa.h, dsa_select).  The fused
     path is fold, indexer/top-k.  Fewer than 80 128-row blocks over more
-    than 2048 keys add one launch: fold, score sweep, radix top-k."""
+    than 2048 keys add one launch: fold, score sweep, histogram top-k."""
     blocks = wl.batch * ((max(wl.seqlens_q) + 127) // 128)
     split = max(wl.seqlens_q) >= 64 and blocks < 80 and max(wl.seqlens_k) > 2048
     return (4 if split else 3)
