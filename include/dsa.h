@@ -294,7 +294,9 @@ DSA_API int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t
  * scales: about 4.3 MB) is a static array inside the library that every GPU
  * loading the library keeps until the process exits.  The first call on a
  * device looks up that array's device address (once per device); make that
- * first call before any stream capture begins.  All calls share the one
+ * first call before any stream capture begins.  The address is kept for the
+ * life of the process: do not call this entry point after a reset of the
+ * device's primary context (cudaDeviceReset) in the same process.  All calls share the one
  * array, so calls whose work overlaps on the GPU (other streams, other host
  * threads) race; serialise them.  The status header is cleared at the start
  * of every call.  The call allocates nothing, waits for `stream` to finish
