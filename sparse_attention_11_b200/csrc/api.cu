@@ -3,11 +3,27 @@
 // Every numeric step runs in the kernels; this file only checks and routes.
 #include <string.h>
 
+#ifndef DSA_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 #include "dsa_kernels.h"
 
 using namespace dsa;
 
 namespace {
+
+// An NVTX range over one entry point (host side: its validation and
+// enqueueing), named after it, for timeline tools; a no-op when no tool is
+// attached, and compiled out with DSA_NO_NVTX.
+struct Range {
+#ifndef DSA_NO_NVTX
+    explicit Range(const char* name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+#else
+    explicit Range(const char*) {}
+#endif
+};
 
 constexpr size_t kHdr = 256;
 constexpr int64_t kTcIndexerMinRows = 64;  // prefill-shaped query sets use the tensor-core indexer
@@ -468,6 +484,7 @@ int dsa_workspace_size(int op, const dsa_seqs* seqs, int32_t k, const dsa_indexe
 
 int dsa_fold(const dsa_seqs* seqs, const dsa_indexer_args* ia, void* u_out, float* s_row_out, void* ws, size_t ws_bytes,
              dsa_stream_t stream) {
+    const Range range("dsa_fold");
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
     if (!r && seqs->total_q && (!u_out || !s_row_out || !aligned(u_out, 16))) r = DSA_ERR_INVALID_ARG;
@@ -478,6 +495,7 @@ int dsa_fold(const dsa_seqs* seqs, const dsa_indexer_args* ia, void* u_out, floa
 
 int dsa_index_scores(const dsa_seqs* seqs, const dsa_indexer_args* ia, int64_t row_begin, int64_t row_count,
                      float* scores, int64_t ld_scores, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_index_scores");
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
     if (r) return r;
@@ -502,6 +520,7 @@ int dsa_index_scores(const dsa_seqs* seqs, const dsa_indexer_args* ia, int64_t r
 
 int dsa_topk(const dsa_seqs* seqs, const float* scores, int64_t ld_scores, int64_t row_begin, int64_t row_count,
              int32_t k, int32_t* idx, int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_topk");
     int r = check_seqs(seqs);
     if (r) return r;
     if (k < 1 || row_begin < 0 || row_count < 0 || row_begin + row_count > seqs->total_q) return DSA_ERR_INVALID_ARG;
@@ -515,6 +534,7 @@ int dsa_sparse_attn_bwd(const dsa_seqs* seqs, const dsa_attn_args* aa, const int
                         int32_t k_sel, const void* d_out, int64_t d_out_stride_tok, int64_t d_out_stride_head,
                         float* d_q, int64_t d_q_stride_tok, int64_t d_q_stride_head, float* d_k, int64_t d_k_stride,
                         float* d_v, int64_t d_v_stride, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_sparse_attn_bwd");
     int r = check_seqs(seqs);
     if (r) return r;
     if (!aa) return DSA_ERR_INVALID_ARG;
@@ -575,6 +595,7 @@ int dsa_sparse_attn_bwd(const dsa_seqs* seqs, const dsa_attn_args* aa, const int
 
 int dsa_attn_target(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel,
                     float* p, int64_t ld_p, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_attn_target");
     int r = check_seqs(seqs);
     if (r) return r;
     if (!aa) return DSA_ERR_INVALID_ARG;
@@ -619,6 +640,7 @@ int dsa_indexer_kl(const dsa_seqs* seqs, const float* q_idx, int64_t q_stride, c
                    int64_t k_stride, const int32_t* idx, int64_t ld_idx, int32_t k_sel, const float* p, int64_t ld_p,
                    float* loss, float* d_q, int64_t d_q_stride, float* d_W, float* d_k, int64_t d_k_stride, void* ws,
                    size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_indexer_kl");
     int r = check_seqs(seqs);
     if (r) return r;
     if (k_sel < 0 || k_sel > 16384 || ld_idx < k_sel || ld_p < k_sel) return DSA_ERR_INVALID_ARG;
@@ -656,6 +678,7 @@ int dsa_indexer_kl(const dsa_seqs* seqs, const float* q_idx, int64_t q_stride, c
 
 int dsa_sparse_attn(const dsa_seqs* seqs, const dsa_attn_args* aa, const int32_t* idx, int64_t ld_idx, int32_t k_sel,
                     void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_sparse_attn");
     int r = check_seqs(seqs);
     if (!r) r = check_attn(seqs, aa);
     if (r) return r;
@@ -692,6 +715,7 @@ int select_into(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int
 
 int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx, int64_t ld_idx, void* ws,
                size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_select");
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
     if (r) return r;
@@ -705,6 +729,7 @@ int dsa_select(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int3
 
 int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k, int32_t* idx_out,
                 int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const Range range("dsa_forward");
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
     if (!r) r = check_attn(seqs, aa);
@@ -727,6 +752,7 @@ int dsa_forward(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn
 int dsa_forward_host(const dsa_seqs* seqs, const dsa_indexer_args* ia, const dsa_attn_args* aa, int32_t k,
                      int32_t* idx_out, int64_t ld_idx, void* ws, size_t ws_bytes, dsa_stream_t stream,
                      dsa_stream_t h2d_stream, dsa_stream_t d2h_stream) {
+    const Range range("dsa_forward_host");
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
     if (!r) r = check_attn(seqs, aa);
@@ -853,6 +879,7 @@ int noalloc_scratch(uint8_t** out) {
 
 extern "C" int dsa_select_noalloc(const dsa_seqs* seqs, const dsa_indexer_args* ia, int32_t k, int32_t* idx,
                                   int64_t ld_idx, dsa_stream_t stream) {
+    const Range range("dsa_select_noalloc");
     int r = check_seqs(seqs);
     if (!r) r = check_indexer(seqs, ia);
     if (r) return r;
